@@ -1,0 +1,173 @@
+/*
+ * bitlinear.h -- C ABI of the B200 (sm_100a) BitNet b1.58 BitLinear library.
+ *
+ * The layer (BitNet b1.58 pages: aratech.ae, "BitNet b1.58: Microsoft's 1-bit
+ * LLM that runs a 100B model on a single CPU", sections "Ternary weights
+ * {-1, 0, +1}" and "BitLinear: the building block"; bhfrc.com/news/56965,
+ * sec. 1.1 and sec. 4.1):
+ *
+ *   gamma   = mean_{n,k} |W_nk|                       (per tensor, fp64 sum)
+ *   code_nk = clip(round(W_nk / (gamma + eps)), -1, 1)            in {-1,0,1}
+ *   s_m     = 127 / max_k |x_mk|                      (per token, fp32)
+ *   q_mk    = clip(rint(x_mk * s_m), -127, 127)                   int8
+ *   acc_mn  = sum_k q_mk * code_nk                                int32
+ *   y_mn    = acc_mn * gamma / s_m                    (fp32, or bf16 output)
+ *
+ * Conventions for every entry point:
+ *   - Every pointer argument is a DEVICE pointer owned by the caller, except
+ *     where a comment says "host".  The library never allocates, frees or
+ *     retains memory; its only global state is one status word per device.
+ *   - Device array pointers must be 16-byte aligned; the single-value
+ *     pointers gamma64 / gamma32 need only their natural alignment
+ *     (BL_ERR_ALIGN otherwise).
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Every call only enqueues work on it and returns; results are
+ *     ready when the stream reaches that point.
+ *   - Arguments are validated on the host before anything is launched; a
+ *     failed check returns its status and enqueues nothing.  A launch failure
+ *     returns BL_ERR_CUDA.
+ *   - Non-finite values met on the device (NaN/Inf in W or x) do not trap:
+ *     they set the device status word, which bitlinear_get_status() returns.
+ *   - Integer accumulation is int32, so K must satisfy 127 * K < 2^31
+ *     (BL_ERR_OVERFLOW otherwise).
+ *   - There is no bias term (the pages show none).
+ */
+#ifndef BITLINEAR_H
+#define BITLINEAR_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    BL_OK = 0,
+    BL_ERR_NULL = 1,        /* a required pointer is NULL                         */
+    BL_ERR_SHAPE = 2,       /* M, N or K out of range                              */
+    BL_ERR_ALIGN = 3,       /* a device pointer is not 16-byte aligned             */
+    BL_ERR_DTYPE = 4,       /* unknown bl_dtype value                              */
+    BL_ERR_WORKSPACE = 5,   /* workspace smaller than the *_workspace_bytes() size */
+    BL_ERR_OVERFLOW = 6,    /* 127 * K >= 2^31: int32 accumulator could overflow   */
+    BL_ERR_NONFINITE = 7,   /* device saw NaN/Inf in W or x (from get_status)      */
+    BL_ERR_CUDA = 8,        /* a CUDA runtime call or kernel launch failed          */
+    BL_ERR_ARG = 9          /* another argument is invalid (eps < 0, count <= 0)   */
+} bl_status;
+
+typedef enum { BL_F32 = 0, BL_BF16 = 1 } bl_dtype;
+
+/* ------------------------------------------------------------------------
+ * Packed ternary weight layout (2 bits per weight, row-tiled, chunk-major).
+ * Code values follow bhfrc.com/news/56965 sec. 4.1: 00 -> 0, 01 -> +1,
+ * 10 -> -1, 11 -> padding (decodes to 0).
+ *   Kp = ceil(K/64)*64, Np = ceil(N/8)*8, C = Kp/64 sixteen-byte chunks/row.
+ *   Weight (n, k) sits in byte  (n/8)*(8*C*16) + ((k/64)*8 + n%8)*16
+ *                                + ((k%64)/16)*4 + k%4
+ *   at bits 2*((k%16)/4) .. +1.  Padded positions (n >= N or k >= K) hold 11.
+ * So each 8-row tile stores chunk c of its 8 rows as 128 contiguous bytes,
+ * and a warp reads 4 chunks x 8 rows as one 512-byte coalesced span.
+ * ---------------------------------------------------------------------- */
+
+/* Padded reduction length Kp = ceil(K/64)*64 (the row stride of q). */
+int64_t bitlinear_padded_k(int64_t K);
+
+/* Bytes of the packed weight buffer: Np * Kp / 4.  Returns 0 if N or K <= 0. */
+int64_t bitlinear_packed_bytes(int64_t N, int64_t K);
+
+/* Bytes of scratch bitlinear_pack_weights needs (fp64 partial sums). */
+int64_t bitlinear_pack_workspace_bytes(int64_t N, int64_t K);
+
+/* ------------------------------------------------------------------------
+ * bitlinear_pack_weights -- absmean quantisation of one weight tensor to
+ * ternary codes and the 2-bit packed layout above (aratech.ae, "Ternary
+ * weights {-1, 0, +1}": scale 1/mean|W|, then clip(-1, 1)(round(.)) ).
+ *
+ *   W         fp32 [N][K] row-major (nn.Linear weight: out x in), device.
+ *   eps       >= 0, added to gamma (fp64) in the code decision only.
+ *   packed    uint8 [bitlinear_packed_bytes(N, K)], device, written.
+ *   gamma64   one double, device, written: mean|W| (fp64 accumulation in a
+ *             fixed, run-to-run deterministic order).
+ *   gamma32   one float, device, written: (float)gamma64, used by forward.
+ *   workspace >= bitlinear_pack_workspace_bytes(N, K) bytes, device scratch.
+ * The code decision |W|/(gamma+eps) > 1/2 is taken exactly (as in fp64).
+ * Errors: NULL, SHAPE (N, K <= 0 or N*K >= 2^40), ALIGN, WORKSPACE, ARG
+ * (eps < 0 or not finite), CUDA.  NaN/Inf in W sets BL_ERR_NONFINITE.
+ * ---------------------------------------------------------------------- */
+bl_status bitlinear_pack_weights(const float* W, int64_t N, int64_t K, double eps,
+                                 uint8_t* packed, double* gamma64, float* gamma32,
+                                 void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * bitlinear_quant_act -- per-token absmax int8 quantisation (aratech.ae,
+ * "BitLinear: the building block": each token's largest |activation| is
+ * mapped to 127).
+ *
+ *   x   [M][K] row-major, fp32 (xt = BL_F32) or bf16 (xt = BL_BF16), device.
+ *   q   int8 [M][Kp] row-major, Kp = bitlinear_padded_k(K), device, written;
+ *       columns K..Kp-1 are written as 0.
+ *   s   fp32 [M], device, written: s_m = 127 / max(max_k |x_mk|, 1e-5).
+ * q_mk = clamp(rint(x_mk * s_m), -127, 127) in fp32 (IEEE divide, no FMA).
+ * Errors: NULL, SHAPE (M, K <= 0), ALIGN, DTYPE, OVERFLOW, CUDA.
+ * ---------------------------------------------------------------------- */
+bl_status bitlinear_quant_act(const void* x, bl_dtype xt, int64_t M, int64_t K, int8_t* q,
+                              float* s, void* stream);
+
+/* ------------------------------------------------------------------------
+ * bitlinear_forward -- ternary x int8 product with int32 accumulation
+ * (bhfrc.com/news/56965 sec. 1.1: each weight adds, subtracts or skips an
+ * activation) and the rescale y = acc * gamma / s.
+ *
+ *   q        int8 [M][Kp] from bitlinear_quant_act, device.
+ *   s        fp32 [M] from bitlinear_quant_act, device.
+ *   packed   from bitlinear_pack_weights (same N, K), device.
+ *   gamma32  one float from bitlinear_pack_weights, device.
+ *   y        [M][N] row-major, fp32 (yt = BL_F32) or bf16 (BL_BF16), device.
+ *   acc_debug  NULL, or int32 [M][N] device buffer that receives acc.
+ * fp32 y equals (float)((double)acc * gamma32 / s_m) for M <= 16 (decode
+ * kernel); the tensor-core kernel (M > 16) evaluates the same product with
+ * a per-token fp64 factor, within 1 fp32 ulp of it.
+ * Errors: NULL, SHAPE (M, N, K <= 0), ALIGN, DTYPE, OVERFLOW, CUDA.
+ * ---------------------------------------------------------------------- */
+bl_status bitlinear_forward(const int8_t* q, const float* s, const uint8_t* packed,
+                            const float* gamma32, int64_t M, int64_t N, int64_t K, void* y,
+                            bl_dtype yt, int32_t* acc_debug, void* stream);
+
+/* ------------------------------------------------------------------------
+ * bitlinear_forward_x -- the same layer with the activation quantisation
+ * fused into the product kernel's prologue: x goes in, y comes out, q and s
+ * never reach memory.  Results are identical to bitlinear_quant_act followed
+ * by bitlinear_forward.  Arguments as in those two calls.
+ * Errors: NULL, SHAPE (M, N, K <= 0; M > 16, or M' * Kp > 160 KiB with M'
+ * = M rounded up to a power of two, for this fused decode form), ALIGN,
+ * DTYPE, OVERFLOW, CUDA.
+ * ---------------------------------------------------------------------- */
+bl_status bitlinear_forward_x(const void* x, bl_dtype xt, const uint8_t* packed,
+                              const float* gamma32, int64_t M, int64_t N, int64_t K, void* y,
+                              bl_dtype yt, void* stream);
+
+/* ------------------------------------------------------------------------
+ * bitlinear_forward_x_grouped -- `count` independent fused BitLinear layers
+ * (the linears of one transformer block) in ONE kernel launch.  Host arrays
+ * of length `count` give each problem's device pointers and sizes, with the
+ * meaning of bitlinear_forward_x.  All problems share M, xt and yt.
+ * Errors: as bitlinear_forward_x, plus ARG (count < 1 or > 16).
+ * ---------------------------------------------------------------------- */
+bl_status bitlinear_forward_x_grouped(int count, const void* const* x, bl_dtype xt,
+                                      const uint8_t* const* packed, const float* const* gamma32,
+                                      int64_t M, const int64_t* N, const int64_t* K,
+                                      void* const* y, bl_dtype yt, void* stream);
+
+/* Synchronises `stream`, then returns and clears the device status word of
+ * the current device: BL_OK, or BL_ERR_NONFINITE if a kernel met NaN/Inf.
+ * Returns BL_ERR_CUDA if the synchronisation itself failed. */
+bl_status bitlinear_get_status(void* stream);
+
+/* Static, human-readable name of a status value (never NULL). */
+const char* bitlinear_status_string(bl_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BITLINEAR_H */

@@ -1,0 +1,206 @@
+// bl_api.cu -- the C ABI of include/bitlinear.h: host-side argument checks,
+// the per-device status word, and dispatch to the kernels.
+#include <cmath>
+#include <cstring>
+
+#include "bl_internal.cuh"
+
+// One status word per device (the only global state of the library).
+__device__ unsigned int g_bl_status_word;
+
+namespace {
+
+constexpr int64_t kMaxK = (int64_t(1) << 31) / 127;   // 127*K must stay < 2^31
+constexpr size_t kFusedSmemLimit = 160 * 1024;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned_to(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+unsigned* status_word()
+{
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_bl_status_word) != cudaSuccess) return nullptr;
+    return static_cast<unsigned*>(p);
+}
+
+int pow2_tokens(int64_t M)
+{
+    return M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : M <= 8 ? 8 : 16;
+}
+
+bl_status check_dtype(bl_dtype t) { return (t == BL_F32 || t == BL_BF16) ? BL_OK : BL_ERR_DTYPE; }
+
+bl_status check_forward_shape(int64_t M, int64_t N, int64_t K)
+{
+    if (M <= 0 || N <= 0 || K <= 0) return BL_ERR_SHAPE;
+    if (M > (int64_t(1) << 31) || N > (int64_t(1) << 31)) return BL_ERR_SHAPE;
+    if (K > kMaxK) return BL_ERR_OVERFLOW;
+    if ((bl::padded_n(N) / 8) > (int64_t(1) << 30)) return BL_ERR_SHAPE;
+    return BL_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int64_t bitlinear_padded_k(int64_t K) { return K <= 0 ? 0 : bl::padded_k(K); }
+
+int64_t bitlinear_packed_bytes(int64_t N, int64_t K)
+{
+    if (N <= 0 || K <= 0) return 0;
+    return bl::padded_n(N) * bl::padded_k(K) / 4;
+}
+
+int64_t bitlinear_pack_workspace_bytes(int64_t N, int64_t K)
+{
+    if (N <= 0 || K <= 0) return 0;
+    return (int64_t)bl::absmean_blocks(N * K) * 8 + 16;
+}
+
+bl_status bitlinear_pack_weights(const float* W, int64_t N, int64_t K, double eps, uint8_t* packed,
+                                 double* gamma64, float* gamma32, void* workspace,
+                                 size_t workspace_bytes, void* stream)
+{
+    if (!W || !packed || !gamma64 || !gamma32 || !workspace) return BL_ERR_NULL;
+    if (N <= 0 || K <= 0 || N > (int64_t(1) << 40) / K) return BL_ERR_SHAPE;
+    if (!aligned16(W) || !aligned16(packed) || !aligned16(workspace) || !aligned_to(gamma64, 8) ||
+        !aligned_to(gamma32, 4))
+        return BL_ERR_ALIGN;
+    if (!(eps >= 0.0) || !std::isfinite(eps)) return BL_ERR_ARG;
+    if ((int64_t)workspace_bytes < bitlinear_pack_workspace_bytes(N, K)) return BL_ERR_WORKSPACE;
+    unsigned* status = status_word();
+    if (!status) return BL_ERR_CUDA;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int64_t count = N * K;
+    const int blocks = bl::absmean_blocks(count);
+    double* partial = static_cast<double*>(workspace);
+    float* thr = reinterpret_cast<float*>(static_cast<char*>(workspace) + (size_t)blocks * 8);
+    if (bl::launch_absmean_partial(W, count, partial, blocks, status, st) != cudaSuccess) return BL_ERR_CUDA;
+    if (bl::launch_absmean_finalize(partial, blocks, count, eps, gamma64, gamma32, thr, st) != cudaSuccess)
+        return BL_ERR_CUDA;
+    if (bl::launch_pack(W, N, K, thr, packed, st) != cudaSuccess) return BL_ERR_CUDA;
+    return BL_OK;
+}
+
+bl_status bitlinear_quant_act(const void* x, bl_dtype xt, int64_t M, int64_t K, int8_t* q, float* s,
+                              void* stream)
+{
+    if (!x || !q || !s) return BL_ERR_NULL;
+    if (check_dtype(xt) != BL_OK) return BL_ERR_DTYPE;
+    if (M <= 0 || K <= 0 || M > (int64_t(1) << 31) - 1) return BL_ERR_SHAPE;
+    if (K > kMaxK) return BL_ERR_OVERFLOW;
+    if (!aligned16(x) || !aligned16(q) || !aligned16(s)) return BL_ERR_ALIGN;
+    unsigned* status = status_word();
+    if (!status) return BL_ERR_CUDA;
+    return bl::launch_quant(x, xt, M, K, q, s, status, static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? BL_OK
+               : BL_ERR_CUDA;
+}
+
+bl_status bitlinear_forward(const int8_t* q, const float* s, const uint8_t* packed,
+                            const float* gamma32, int64_t M, int64_t N, int64_t K, void* y,
+                            bl_dtype yt, int32_t* acc_debug, void* stream)
+{
+    if (!q || !s || !packed || !gamma32 || !y) return BL_ERR_NULL;
+    if (check_dtype(yt) != BL_OK) return BL_ERR_DTYPE;
+    bl_status st = check_forward_shape(M, N, K);
+    if (st != BL_OK) return st;
+    if (!aligned16(q) || !aligned16(s) || !aligned16(packed) || !aligned_to(gamma32, 4) || !aligned16(y) ||
+        (acc_debug && !aligned16(acc_debug)))
+        return BL_ERR_ALIGN;
+    unsigned* status = status_word();
+    if (!status) return BL_ERR_CUDA;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    if (M > bl::kFusedMaxM && bl::gemm_tc_supported(M, N, K))
+        return bl::launch_gemm_tc(q, s, packed, gamma32, M, N, K, y, yt, acc_debug, cs) == cudaSuccess
+                   ? BL_OK
+                   : BL_ERR_CUDA;
+    bl::GemvBatch b;
+    std::memset(&b, 0, sizeof(b));
+    b.count = 1;
+    b.M = M;
+    b.p[0].q = q;
+    b.p[0].s = s;
+    b.p[0].packed = packed;
+    b.p[0].gamma32 = gamma32;
+    b.p[0].y = y;
+    b.p[0].acc = acc_debug;
+    b.p[0].N = N;
+    b.p[0].K = K;
+    return bl::launch_gemv(b, false, BL_F32, yt, status, cs) == cudaSuccess ? BL_OK : BL_ERR_CUDA;
+}
+
+bl_status bitlinear_forward_x_grouped(int count, const void* const* x, bl_dtype xt,
+                                      const uint8_t* const* packed, const float* const* gamma32,
+                                      int64_t M, const int64_t* N, const int64_t* K, void* const* y,
+                                      bl_dtype yt, void* stream)
+{
+    if (count < 1 || count > bl::kMaxGroup) return BL_ERR_ARG;
+    if (!x || !packed || !gamma32 || !N || !K || !y) return BL_ERR_NULL;
+    if (check_dtype(xt) != BL_OK || check_dtype(yt) != BL_OK) return BL_ERR_DTYPE;
+    if (M <= 0 || M > bl::kFusedMaxM) return BL_ERR_SHAPE;
+    bl::GemvBatch b;
+    std::memset(&b, 0, sizeof(b));
+    b.count = count;
+    b.M = M;
+    int64_t tiles = 0;
+    for (int i = 0; i < count; ++i) {
+        if (!x[i] || !packed[i] || !gamma32[i] || !y[i]) return BL_ERR_NULL;
+        bl_status st = check_forward_shape(M, N[i], K[i]);
+        if (st != BL_OK) return st;
+        if ((size_t)pow2_tokens(M) * (size_t)bl::padded_k(K[i]) > kFusedSmemLimit) return BL_ERR_SHAPE;
+        if (!aligned16(x[i]) || !aligned16(packed[i]) || !aligned_to(gamma32[i], 4) || !aligned16(y[i]))
+            return BL_ERR_ALIGN;
+        tiles += bl::padded_n(N[i]) / 8;
+        b.p[i].x = x[i];
+        b.p[i].packed = packed[i];
+        b.p[i].gamma32 = gamma32[i];
+        b.p[i].y = y[i];
+        b.p[i].N = N[i];
+        b.p[i].K = K[i];
+    }
+    if (tiles > (int64_t(1) << 31) - 1) return BL_ERR_SHAPE;
+    unsigned* status = status_word();
+    if (!status) return BL_ERR_CUDA;
+    return bl::launch_gemv(b, true, xt, yt, status, static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? BL_OK
+               : BL_ERR_CUDA;
+}
+
+bl_status bitlinear_forward_x(const void* x, bl_dtype xt, const uint8_t* packed, const float* gamma32,
+                              int64_t M, int64_t N, int64_t K, void* y, bl_dtype yt, void* stream)
+{
+    return bitlinear_forward_x_grouped(1, &x, xt, &packed, &gamma32, M, &N, &K, &y, yt, stream);
+}
+
+bl_status bitlinear_get_status(void* stream)
+{
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return BL_ERR_CUDA;
+    unsigned v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_bl_status_word, sizeof(v)) != cudaSuccess) return BL_ERR_CUDA;
+    if (v != 0) {
+        const unsigned zero = 0;
+        if (cudaMemcpyToSymbol(g_bl_status_word, &zero, sizeof(zero)) != cudaSuccess) return BL_ERR_CUDA;
+        return BL_ERR_NONFINITE;
+    }
+    return BL_OK;
+}
+
+const char* bitlinear_status_string(bl_status status)
+{
+    switch (status) {
+        case BL_OK: return "BL_OK";
+        case BL_ERR_NULL: return "BL_ERR_NULL: a required pointer is NULL";
+        case BL_ERR_SHAPE: return "BL_ERR_SHAPE: M, N or K out of range";
+        case BL_ERR_ALIGN: return "BL_ERR_ALIGN: a device pointer is not 16-byte aligned";
+        case BL_ERR_DTYPE: return "BL_ERR_DTYPE: unknown dtype";
+        case BL_ERR_WORKSPACE: return "BL_ERR_WORKSPACE: workspace too small";
+        case BL_ERR_OVERFLOW: return "BL_ERR_OVERFLOW: 127*K >= 2^31, int32 accumulator could overflow";
+        case BL_ERR_NONFINITE: return "BL_ERR_NONFINITE: NaN or Inf met in W or x";
+        case BL_ERR_CUDA: return "BL_ERR_CUDA: a CUDA call or kernel launch failed";
+        case BL_ERR_ARG: return "BL_ERR_ARG: invalid argument";
+    }
+    return "unknown bl_status";
+}
+
+}  // extern "C"

@@ -1,0 +1,76 @@
+// bl_internal.cuh -- private declarations shared by the library's .cu files.
+//
+// Nothing here is part of the C ABI (include/bitlinear.h is).  The packed
+// weight layout constants below restate that header's layout spec.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "../../include/bitlinear.h"
+
+namespace bl {
+
+// ---- packed layout (include/bitlinear.h) -------------------------------
+constexpr int kTileRows = 8;        // rows per tile
+constexpr int kChunkK = 64;         // weights per 16-byte chunk
+constexpr int kChunkBytes = 16;
+
+__host__ __device__ inline int64_t padded_k(int64_t K) { return (K + 63) / 64 * 64; }
+__host__ __device__ inline int64_t padded_n(int64_t N) { return (N + 7) / 8 * 8; }
+__host__ __device__ inline int64_t chunks_per_row(int64_t K) { return padded_k(K) / 64; }
+// bytes of one 8-row tile
+__host__ __device__ inline int64_t tile_bytes(int64_t K) { return chunks_per_row(K) * 8 * 16; }
+
+// ---- device status word bits --------------------------------------------
+constexpr unsigned kStatusNonfiniteW = 1u;
+constexpr unsigned kStatusNonfiniteX = 2u;
+
+// ---- launch helpers (host side, one per .cu file) ------------------------
+// Each returns cudaSuccess or the launch error; validation is done by the
+// caller in bl_api.cu.
+cudaError_t launch_absmean_partial(const float* W, int64_t count, double* partial, int blocks,
+                                   unsigned* status, cudaStream_t st);
+cudaError_t launch_absmean_finalize(const double* partial, int blocks, int64_t count, double eps,
+                                    double* gamma64, float* gamma32, float* thr, cudaStream_t st);
+cudaError_t launch_pack(const float* W, int64_t N, int64_t K, const float* thr, uint8_t* packed,
+                        cudaStream_t st);
+int absmean_blocks(int64_t count);
+
+cudaError_t launch_quant(const void* x, bl_dtype xt, int64_t M, int64_t K, int8_t* q, float* s,
+                         unsigned* status, cudaStream_t st);
+
+// One problem of the decode kernel (packed ternary x int8 -> y).
+struct GemvProblem {
+    const void* x;          // fused form: activations [M][K] (fp32/bf16)
+    const int8_t* q;        // unfused form: int8 [M][Kp]
+    const float* s;         // unfused form: fp32 [M]
+    const uint8_t* packed;  // packed ternary weights
+    const float* gamma32;   // per-tensor scale
+    void* y;                // [M][N]
+    int32_t* acc;           // optional int32 [M][N]
+    int64_t N, K;
+    int64_t tile_begin;     // first 8-row tile index of this problem in the grid
+};
+constexpr int kMaxGroup = 16;
+struct GemvBatch {
+    GemvProblem p[kMaxGroup];
+    int count;
+    int64_t M;
+};
+
+cudaError_t launch_gemv(const GemvBatch& b, bool fused, bl_dtype xt, bl_dtype yt, unsigned* status,
+                        cudaStream_t st);
+// Largest M the fused decode kernel accepts.
+constexpr int kFusedMaxM = 16;
+
+// Prefill tensor-core GEMM (tcgen05 kind::i8).  Returns cudaErrorNotSupported
+// when the shape is outside what the kernel handles; the caller then uses
+// the decode kernel.
+cudaError_t launch_gemm_tc(const int8_t* q, const float* s, const uint8_t* packed,
+                           const float* gamma32, int64_t M, int64_t N, int64_t K, void* y,
+                           bl_dtype yt, int32_t* acc, cudaStream_t st);
+bool gemm_tc_supported(int64_t M, int64_t N, int64_t K);
+
+}  // namespace bl
