@@ -1,20 +1,24 @@
 #!/usr/bin/env python3
 """Benchmark of the BitNet b1.58 BitLinear hot path on B200.
 
-Default workload (N=1 line): decode, M = 1 token, through the seven linears
-of a 2B-class block (2560->6912 x2, 6912->2560, 2560->2560 x2, 2560->640
-x2), x bf16 ~ N(0,1) with 1% outliers x20, fp32 y.  One step = one pass of
-the per-token hot path over the block: per-token absmax int8 quantisation,
-ternary x int8 product with int32 accumulation and the rescale, for all
-seven linears (the weights are packed once, before timing, as a model's
-weights are).  Metric: algorithmic bytes (packed weights N*K/4 + bf16 x +
-fp32 y) per second.
+Default workload (the N=1 line): decode, M = 1 token, through the seven
+linears of a 2B-class block (2560->6912 x2, 6912->2560, 2560->2560 x2,
+2560->640 x2), x bf16 ~ N(0,1) with 1% outliers x20, fp32 y.  One step is
+one pass of the per-token hot path over the block: per-token absmax int8
+quantisation, ternary x int8 product with int32 accumulation and the
+rescale, for all seven linears (weights are packed once beforehand, as a
+model's weights are; packing is timed separately).  Metric: algorithmic
+bytes (packed weights N*K/4 + bf16 x + fp32 y) per second.
 
-The packed weights of the block are replicated into enough copies that the
-rotating working set exceeds 3x the L2 size, so every step streams its
-weights from HBM.  Steps are replayed from CUDA graphs and timed with CUDA
-events on the launching stream; multi-GPU runs are independent replicas
-(no collective on the data path) timed as the max over ranks.
+The packed weights are replicated into enough copies that the rotating
+working set exceeds 3x the L2 size, so every step streams its weights from
+HBM.  Steps are replayed from CUDA graphs and timed with CUDA events on the
+launching stream; multi-GPU runs are independent replicas (no collective on
+the data path), timed as the max over ranks.
+
+Other workloads (--workload): 7b (decode at 7B-class shapes, --m 1/4/16),
+prefill (M = 2048 tokens on the tensor cores; metric int8 TOPS), pack
+(absmean quantise + 2-bit pack of the block's weights).
 
 --impl reference times the CPU oracle (oracle/, plain C) on the same
 workload and metric, on this machine's host cores.
@@ -35,6 +39,7 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "BitLinear decode weight GB/s (% of HBM peak); prefill int8 TOPS (% peak)"
+NOMINAL_INT8_OVER_BF16 = 2.0     # dense int8 / dense bf16 tensor throughput (4.5 / 2.25 PFLOP/s)
 
 
 def parse_args():
@@ -43,12 +48,15 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=4000)
     ap.add_argument("--warmup", type=int, default=200)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=["block2b", "7b", "prefill", "pack"], default="block2b")
+    ap.add_argument("--m", type=int, default=1, help="tokens for --workload 7b")
     ap.add_argument("--mode", choices=["grouped", "fused", "separate"], default="grouped",
-                    help="grouped: one launch per step; fused: one launch per linear; "
-                         "separate: quantise + product launches per linear")
+                    help="decode: grouped = one launch per step; fused = one launch per linear; "
+                         "separate = quantise + product launches per linear")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="oracle CPU-baseline budget")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true", help="skip the prefill sub-measurement")
     return ap.parse_args()
 
 
@@ -58,8 +66,10 @@ def load_peaks():
     if os.path.exists(p):
         with open(p) as f:
             d = json.load(f)
-        return float(d["hbm_gbs"]), "measured"
-    return 6650.0, "fallback"
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "kind": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "kind": "fallback"}
 
 
 class ClockSampler:
@@ -118,96 +128,388 @@ class ClockSampler:
                 "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(self.samples)}
 
 
-def block_bytes(lin, M):
-    """Algorithmic bytes of one pass over the block: packed W + bf16 x + fp32 y."""
+def decode_bytes(lin, M):
+    """Algorithmic bytes of one decode pass: packed W + bf16 x + fp32 y."""
     return sum(L["N"] * L["K"] // 4 + M * L["K"] * 2 + M * L["N"] * 4 for L in lin)
 
 
+def max_over_ranks(ms, dist, dev):
+    if dist is None:
+        return ms
+    import torch
+    t = torch.tensor([ms], device=dev, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def linears_for(args):
+    import synth
+    if args.workload == "7b":
+        M = args.m
+        lin = []
+        for i, (K, N, name) in enumerate(synth.SHAPES_7B):
+            lin.append(dict(name=name, K=K, N=N, W=synth.weights(N, K, 10 + i),
+                            x=synth.activations(M, K, 2000 + i, "bf16")))
+        return lin, M, f"7b_decode_m{M}"
+    if args.workload == "prefill":
+        M = synth.M_PREFILL
+        lin = []
+        for i, (K, N, name) in enumerate(synth.PREFILL):
+            lin.append(dict(name=name, K=K, N=N, W=synth.weights(N, K, 20 + i),
+                            x=synth.activations(M, K, 3000 + i, "bf16")))
+        return lin, M, "prefill_m2048"
+    return synth.block2b_inputs(seed_base=0, M=1), 1, "block2b_decode_m1"
+
+
 # ----------------------------------------------------- CPU (oracle) arm
-def oracle_block_setup(lin):
+def oracle_setup(lin):
+    import numpy as np
     import oracle
     prepared = []
     for L in lin:
         g64 = oracle.absmean_gamma(L["W"])
         code, _, _ = oracle.ternary_codes(L["W"], g64, 1e-5)
-        prepared.append(dict(x=L["x"], code=code, g32=float(__import__("numpy").float32(g64)), N=L["N"], K=L["K"]))
+        prepared.append(dict(x=L["x"], code=code, g32=float(np.float32(g64)), N=L["N"], K=L["K"]))
     return prepared
 
 
-def oracle_block_pass(prepared, threads, row_frac=1.0):
-    """One oracle pass over the block (quantise, multiply, rescale); with
-    row_frac < 1 only the first row_frac of each weight's rows."""
+def oracle_pass(prepared, threads, row_frac=1.0):
+    """One oracle pass over the linears (quantise, multiply, rescale); with
+    row_frac < 1 only the first row_frac of each weight's output rows.
+    Returns (algorithmic bytes, int ops) of the work done."""
     import oracle
-    nbytes = 0
+    nbytes, ops = 0, 0
     for P in prepared:
         n = max(1, int(P["N"] * row_frac))
         oracle.forward_bf16_mt(P["x"], P["code"][:n], P["g32"], threads)
-        nbytes += n * P["K"] // 4 + P["x"].size * 2 + P["x"].shape[0] * n * 4
-    return nbytes
+        M = P["x"].shape[0]
+        nbytes += n * P["K"] // 4 + P["x"].size * 2 + M * n * 4
+        ops += 2 * M * n * P["K"]
+    return nbytes, ops
 
 
-def cpu_baseline(lin, seconds):
-    prepared = oracle_block_setup(lin)
+def cpu_baseline(lin, seconds, prefill=False):
+    prepared = oracle_setup(lin)
     threads = os.cpu_count() or 1
     t0 = time.perf_counter()
     total, passes = 0, 0
+    frac = 1.0
+    if prefill:   # a full prefill pass is minutes of scalar CPU work: sample rows
+        frac = 0.01
     while True:
-        total += oracle_block_pass(prepared, threads)
+        b, o = oracle_pass(prepared, threads, frac)
+        total += o if prefill else b
         passes += 1
         el = time.perf_counter() - t0
         if el >= seconds:
             break
+    if prefill:
+        return {"value": total / el / 1e12, "unit": "TOPS", "cores": threads, "kind": "oracle",
+                "sample": f"{passes} oracle passes over 1% of the output rows of each prefill linear "
+                          f"({el:.1f} s, {threads} threads)"}
     return {"value": total / el / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
-            "sample": f"{passes} full oracle passes over the 7-linear block at M=1 "
+            "sample": f"{passes} full oracle passes over the linears at M={lin[0]['x'].shape[0]} "
                       f"({el:.1f} s, {threads} threads, rows split across threads)"}
 
 
 def run_reference(args, lin, M, config):
     """The oracle as the reference arm: rank 0 only."""
-    import numpy as np  # noqa: F401
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return None
-    prepared = oracle_block_setup(lin)
+    prefill = args.workload == "prefill"
+    prepared = oracle_setup(lin)
     threads = os.cpu_count() or 1
+    probe = 0.01 if prefill else 1.0
     t0 = time.perf_counter()
-    oracle_block_pass(prepared, threads)
-    t_full = time.perf_counter() - t0
+    oracle_pass(prepared, threads, probe)
+    t_probe = (time.perf_counter() - t0) / probe
     budget = 120.0
-    frac = min(1.0, budget / max(1e-9, t_full * (args.steps + args.warmup)))
+    frac = min(1.0, budget / max(1e-9, t_probe * (args.steps + args.warmup)))
     for _ in range(args.warmup):
-        oracle_block_pass(prepared, threads, frac)
+        oracle_pass(prepared, threads, frac)
     t0 = time.perf_counter()
-    nbytes = 0
+    nbytes, ops = 0, 0
     for _ in range(args.steps):
-        nbytes += oracle_block_pass(prepared, threads, frac)
+        b, o = oracle_pass(prepared, threads, frac)
+        nbytes += b
+        ops += o
     el = time.perf_counter() - t0
-    value = nbytes / el / 1e9
+    value, unit = (ops / el / 1e12, "TOPS") if prefill else (nbytes / el / 1e9, "GB/s")
     sample = (f"each step: oracle pass over {frac * 100:.3g}% of every linear's output rows "
               f"(quantise + multiply + rescale), {threads} threads")
-    return {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": unit, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int64",
             "data": "synthetic", "config": config,
-            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads, "kind": "oracle", "sample": sample},
-            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+            "cpu_baseline": {"value": value, "unit": unit, "cores": threads, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
 # --------------------------------------------------------------- GPU arm
+class Graphs:
+    """CUDA graphs of `copies` consecutive steps and of single steps."""
+
+    def __init__(self, torch, stream, step, copies):
+        self.copies = copies
+        with torch.cuda.stream(stream):
+            self.all = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(self.all, stream=stream):
+                for i in range(copies):
+                    step(i)
+            self.one = []
+            for i in range(copies):
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=stream):
+                    step(i)
+                self.one.append(g)
+
+    def run(self, n):
+        full, rem = divmod(n, self.copies)
+        for _ in range(full):
+            self.all.replay()
+        for i in range(rem):
+            self.one[i].replay()
+
+
+def time_region(torch, stream, fn, dist, dev):
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    e0.record(stream)
+    fn()
+    e1.record(stream)
+    e1.synchronize()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    return max_over_ranks(e0.elapsed_time(e1), dist, dev)
+
+
+def setup_problems(torch, bl, lin, M, dev, want_bytes, out_dtype):
+    """Packs every weight once (GPU packer), then replicates weights, x and y
+    into `copies` sets so that one pass over all copies touches > want_bytes."""
+    import numpy as np
+    packed0, g32s = [], []
+    for L in lin:
+        p, _, g = bl.pack(torch.from_numpy(L["W"]).to(dev))
+        packed0.append(p)
+        g32s.append(g)
+    torch.cuda.synchronize()
+    if bl.bitlinear_get_status() != bl.BL_OK:
+        raise RuntimeError("non-finite weights")
+    per_copy = sum(p.numel() for p in packed0) + sum(M * L["K"] * 2 + M * L["N"] * 4 for L in lin)
+    copies = max(2, math.ceil(want_bytes / per_copy))
+    packed = [[p.clone() for p in packed0] for _ in range(copies)]
+    xs = [[torch.from_numpy(L["x"].view(np.int16)).to(dev).view(torch.bfloat16) for L in lin]
+          for _ in range(copies)]
+    ys = [[torch.empty((M, L["N"]), dtype=out_dtype, device=dev) for L in lin] for _ in range(copies)]
+    return dict(packed=packed, g32=g32s, xs=xs, ys=ys, copies=copies, per_copy=per_copy,
+                Ns=[L["N"] for L in lin], Ks=[L["K"] for L in lin])
+
+
+def run_decode(torch, bl, args, lin, M, dev, stream, dist, l2):
+    S = setup_problems(torch, bl, lin, M, dev, 3 * l2, torch.float32)
+    copies, Ns, Ks = S["copies"], S["Ns"], S["Ks"]
+    mode = args.mode
+    if mode == "grouped" and any(bl_fused_too_big(bl, M, K) for K in Ks):
+        mode = "separate"
+    qs = [torch.empty((M, bl.bitlinear_padded_k(K)), dtype=torch.int8, device=dev) for K in Ks]
+    ss = [torch.empty(M, dtype=torch.float32, device=dev) for _ in Ks]
+
+    def step(i):
+        c = i % copies
+        if mode == "grouped":
+            bl.bitlinear_forward_x_grouped(S["xs"][c], S["packed"][c], S["g32"], Ns, Ks, S["ys"][c], stream)
+            return 1
+        if mode == "fused":
+            for j in range(len(lin)):
+                bl.bitlinear_forward_x(S["xs"][c][j], S["packed"][c][j], S["g32"][j], Ns[j], Ks[j],
+                                       S["ys"][c][j], stream)
+            return len(lin)
+        for j in range(len(lin)):
+            bl.bitlinear_quant_act(S["xs"][c][j], qs[j], ss[j], stream)
+            bl.bitlinear_forward(qs[j], ss[j], S["packed"][c][j], S["g32"][j], M, Ns[j], Ks[j],
+                                 S["ys"][c][j], None, stream)
+        return 2 * len(lin)
+
+    launches = step(0)
+    torch.cuda.synchronize()
+    G = Graphs(torch, stream, step, copies)
+    G.run(max(3, args.warmup))
+    sampler = ClockSampler(dev.index)
+    sampler.start()
+    ms = time_region(torch, stream, lambda: G.run(args.steps), dist, dev)
+    clocks = sampler.stop()
+    if bl.bitlinear_get_status() != bl.BL_OK:
+        raise RuntimeError("device status word set during the timed region")
+    nbytes = decode_bytes(lin, M)
+
+    # dominant kernel: the product kernel (the whole step in grouped mode)
+    if mode == "grouped":
+        kern_ms, kern_bytes, kname = ms / args.steps, nbytes, "stream_kernel (fused quantise, 7 linears, 1 launch)"
+    else:
+        def kstep(i):
+            c = i % copies
+            for j in range(len(lin)):
+                if mode == "fused":
+                    bl.bitlinear_forward_x(S["xs"][c][j], S["packed"][c][j], S["g32"][j], Ns[j], Ks[j],
+                                           S["ys"][c][j], stream)
+                else:
+                    bl.bitlinear_forward(qs[j], ss[j], S["packed"][c][j], S["g32"][j], M, Ns[j], Ks[j],
+                                         S["ys"][c][j], None, stream)
+        GK = Graphs(torch, stream, kstep, copies)
+        GK.run(copies)
+        reps = max(copies, args.steps)
+        kms = time_region(torch, stream, lambda: GK.run(reps), dist, dev)
+        kern_ms = kms / (reps * len(lin))
+        kern_bytes = nbytes / len(lin)
+        kname = "stream_kernel (product, one launch per linear)"
+    return dict(S=S, mode=mode, ms=ms, launches=launches, clocks=clocks, nbytes=nbytes,
+                kern_ms=kern_ms, kern_bytes=kern_bytes, kname=kname)
+
+
+def bl_fused_too_big(bl, M, K):
+    p2 = 1 if M <= 1 else 2 if M <= 2 else 4 if M <= 4 else 8 if M <= 8 else 16
+    return M > 16 or p2 * bl.bitlinear_padded_k(K) > 160 * 1024
+
+
+def run_e2e(torch, bl, lin, M, dev, stream, S, steps, dist):
+    """Pinned host x -> H2D -> grouped C-ABI call -> D2H y, every step."""
+    import numpy as np
+    Ns, Ks, copies = S["Ns"], S["Ks"], S["copies"]
+    hx = torch.empty(sum(M * K for K in Ks), dtype=torch.bfloat16).pin_memory()
+    hy = torch.empty(sum(M * N for N in Ns), dtype=torch.float32).pin_memory()
+    off = 0
+    for L in lin:
+        hx[off:off + M * L["K"]].copy_(torch.from_numpy(L["x"].view(np.int16).ravel()).view(torch.bfloat16))
+        off += M * L["K"]
+    dx = torch.empty_like(hx, device=dev)
+    dy = torch.empty_like(hy, device=dev)
+    xv, yv, ox, oy = [], [], 0, 0
+    for K, N in zip(Ks, Ns):
+        xv.append(dx[ox:ox + M * K].view(M, K))
+        yv.append(dy[oy:oy + M * N].view(M, N))
+        ox += M * K
+        oy += M * N
+
+    def e2e_step(i):
+        dx.copy_(hx, non_blocking=True)
+        bl.bitlinear_forward_x_grouped(xv, S["packed"][i % copies], S["g32"], Ns, Ks, yv, stream)
+        hy.copy_(dy, non_blocking=True)
+
+    for i in range(3):
+        e2e_step(i)
+    n = max(1, min(steps, 2000))
+    ems = time_region(torch, stream, lambda: [e2e_step(i) for i in range(n)], dist, dev)
+    return ems, n, hx.numel() * hx.element_size(), hy.numel() * hy.element_size()
+
+
+def run_prefill(torch, bl, args, dev, stream, dist, l2, steps):
+    import synth
+    lin = []
+    for i, (K, N, name) in enumerate(synth.PREFILL):
+        lin.append(dict(name=name, K=K, N=N, W=synth.weights(N, K, 20 + i),
+                        x=synth.activations(synth.M_PREFILL, K, 3000 + i, "bf16")))
+    M = synth.M_PREFILL
+    S = setup_problems(torch, bl, lin, M, dev, 3 * l2, torch.bfloat16)
+    copies, Ns, Ks = S["copies"], S["Ns"], S["Ks"]
+    qs = [[torch.empty((M, bl.bitlinear_padded_k(K)), dtype=torch.int8, device=dev) for K in Ks]
+          for _ in range(copies)]
+    ss = [[torch.empty(M, dtype=torch.float32, device=dev) for _ in Ks] for _ in range(copies)]
+
+    def step(i):
+        c = i % copies
+        for j in range(len(lin)):
+            bl.bitlinear_quant_act(S["xs"][c][j], qs[c][j], ss[c][j], stream)
+            bl.bitlinear_forward(qs[c][j], ss[c][j], S["packed"][c][j], S["g32"][j], M, Ns[j], Ks[j],
+                                 S["ys"][c][j], None, stream)
+
+    def gstep(i):
+        c = i % copies
+        for j in range(len(lin)):
+            bl.bitlinear_forward(qs[c][j], ss[c][j], S["packed"][c][j], S["g32"][j], M, Ns[j], Ks[j],
+                                 S["ys"][c][j], None, stream)
+
+    step(0)
+    torch.cuda.synchronize()
+    G = Graphs(torch, stream, step, copies)
+    GK = Graphs(torch, stream, gstep, copies)
+    G.run(max(3, min(args.warmup, 20)))
+    ms = time_region(torch, stream, lambda: G.run(steps), dist, dev)
+    GK.run(copies)
+    kms = time_region(torch, stream, lambda: GK.run(steps), dist, dev)
+    ops = sum(2 * M * N * K for N, K in zip(Ns, Ks))
+    peaks = load_peaks()
+    int8_peak = peaks["bf16_tflops"] * NOMINAL_INT8_OVER_BF16
+    achieved = ops / (kms / steps / 1e3) / 1e12
+    # measured int8 ceiling of the library GEMM (cuBLASLt via torch._int_mm), context only
+    ref_tops = None
+    try:
+        a = torch.randint(-127, 128, (8192, 8192), dtype=torch.int8, device=dev)
+        b = torch.randint(-127, 128, (8192, 8192), dtype=torch.int8, device=dev)
+        for _ in range(3):
+            torch._int_mm(a, b)
+        n = 10
+        tms = time_region(torch, stream, lambda: [torch._int_mm(a, b) for _ in range(n)], None, dev)
+        ref_tops = 2 * 8192 ** 3 / (tms / n / 1e3) / 1e12
+        del a, b
+    except Exception:
+        pass
+    return {"workload": "prefill_m2048 (2560->6912, 6912->2560), bf16 x, bf16 y",
+            "value": ops / (ms / steps / 1e3) / 1e12, "unit": "TOPS", "ms_per_step": ms / steps,
+            "steps": steps, "launches_per_step": 2 * len(lin),
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": int8_peak, "unit": "TFLOP/s",
+                         "frac": achieved / int8_peak, "traffic": None,
+                         "kernel": "gemm_tc_kernel (tcgen05 kind::i8, weights expanded into TMEM)",
+                         "peak_kind": f"{peaks['kind']} bf16 burst x nominal int8/bf16 ratio 2",
+                         "avg_launch_us": kms / steps / len(lin) * 1e3,
+                         "cublaslt_int8_8192cubed_tops": ref_tops},
+            "l2_policy": f"{copies} rotating copies of x, q, weights and y (> 3x L2)"}
+
+
+def run_pack(torch, bl, args, dev, stream, dist, l2):
+    import synth
+    lin = synth.block2b_inputs(0, 1)
+    Ws = [torch.from_numpy(L["W"]).to(dev) for L in lin]
+    wbytes = sum(w.numel() * 4 for w in Ws)
+    copies = max(1, math.ceil(3 * l2 / wbytes))
+    Wc = [[w.clone() for w in Ws] for _ in range(copies)]
+    outs = [(torch.empty(bl.bitlinear_packed_bytes(L["N"], L["K"]), dtype=torch.uint8, device=dev),
+             torch.empty(1, dtype=torch.float64, device=dev), torch.empty(1, dtype=torch.float32, device=dev),
+             torch.empty(bl.bitlinear_pack_workspace_bytes(L["N"], L["K"]), dtype=torch.uint8, device=dev))
+            for L in lin]
+
+    def step(i):
+        for j, L in enumerate(lin):
+            p, g64, g32, ws = outs[j]
+            bl.bitlinear_pack_weights(Wc[i % copies][j], 1e-5, p, g64, g32, ws, stream)
+
+    step(0)
+    torch.cuda.synchronize()
+    G = Graphs(torch, stream, step, copies)
+    G.run(3)
+    steps = max(copies, min(args.steps, 200))
+    ms = time_region(torch, stream, lambda: G.run(steps), dist, dev)
+    nweights = sum(L["N"] * L["K"] for L in lin)
+    algo = nweights * 4 + nweights // 4   # read fp32 W once + write 2-bit codes
+    return {"value": algo * steps / (ms / 1e3) / 1e9, "unit": "GB/s", "ms_per_step": ms / steps,
+            "steps": steps, "algorithmic_bytes_per_step": algo, "launches_per_step": 3 * len(lin),
+            "note": "two passes over W (absmean, then codes); the second is served from L2 "
+                    "for weights that fit there"}
+
+
 def main():
     args = parse_args()
-    import numpy as np
-    import synth
-
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
-    M = 1
-    lin = synth.block2b_inputs(seed_base=0, M=M)
-    config = {"workload": "block2b_decode_m1", "M": M,
-              "linears": [f"{L['name']}:{L['K']}->{L['N']}" for L in lin],
-              "x": "bf16 N(0,1), 1% outliers x20", "y": "fp32", "weights": "N(0,0.02) fp32, packed 2-bit",
-              "parallelism": "replicas" if world > 1 else "single"}
+    lin, M, wname = linears_for(args)
+    config = {"workload": wname, "M": M, "linears": [f"{L['name']}:{L['K']}->{L['N']}" for L in lin],
+              "x": "bf16 N(0,1)" + (", 1% outliers x20" if args.workload == "block2b" else ""),
+              "y": "bf16" if args.workload == "prefill" else "fp32",
+              "weights": "N(0,0.02) fp32, packed 2-bit", "parallelism": "replicas" if world > 1 else "single"}
 
     if args.impl == "reference":
         out = run_reference(args, lin, M, config)
@@ -219,7 +521,6 @@ def main():
     import ternary_weight_linear_absmean_b200 as bl
     from ternary_weight_linear_absmean_b200 import _build
     _build.build()
-
     torch.cuda.set_device(local)
     dist = None
     if world > 1:
@@ -230,185 +531,60 @@ def main():
     dev = torch.device("cuda", local)
     stream = torch.cuda.Stream(device=dev)
     torch.cuda.set_stream(stream)
-
-    # ---- pack the block's weights once, then replicate to > 3x L2
-    packed0, g32s = [], []
-    for L in lin:
-        p, _, g = bl.pack(torch.from_numpy(L["W"]).to(dev))
-        packed0.append(p)
-        g32s.append(g)
-    torch.cuda.synchronize()
-    if bl.bitlinear_get_status() != bl.BL_OK:
-        raise RuntimeError("non-finite weights")
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
-    wbytes = sum(p.numel() for p in packed0)
-    copies = max(2, math.ceil(3 * l2 / wbytes))
-    packed = [[p.clone() for p in packed0] for _ in range(copies)]
-    xs = [[torch.from_numpy(L["x"].view(np.int16)).to(dev).view(torch.bfloat16) for L in lin] for _ in range(copies)]
-    ys = [[torch.empty((M, L["N"]), dtype=torch.float32, device=dev) for L in lin] for _ in range(copies)]
-    Ns = [L["N"] for L in lin]
-    Ks = [L["K"] for L in lin]
-    qs = [torch.empty((M, bl.bitlinear_padded_k(K)), dtype=torch.int8, device=dev) for K in Ks]
-    ss = [torch.empty(M, dtype=torch.float32, device=dev) for _ in Ks]
-    config.update({"weight_copies": copies, "rotating_weight_bytes": wbytes * copies,
-                   "l2_bytes": l2, "l2_policy": "inputs larger than L2: weights rotate over copies > 3x L2",
-                   "mode": args.mode})
+    peaks = load_peaks()
 
-    def step(i):
-        c = i % copies
-        if args.mode == "grouped":
-            bl.bitlinear_forward_x_grouped(xs[c], packed[c], g32s, Ns, Ks, ys[c], stream)
-            return 1
-        if args.mode == "fused":
-            for j in range(len(lin)):
-                bl.bitlinear_forward_x(xs[c][j], packed[c][j], g32s[j], Ns[j], Ks[j], ys[c][j], stream)
-            return len(lin)
-        for j in range(len(lin)):
-            bl.bitlinear_quant_act(xs[c][j], qs[j], ss[j], stream)
-            bl.bitlinear_forward(qs[j], ss[j], packed[c][j], g32s[j], M, Ns[j], Ks[j], ys[c][j], None, stream)
-        return 2 * len(lin)
-
-    launches_per_step = step(0)
-    torch.cuda.synchronize()
-
-    # ---- CUDA graphs: one of `copies` steps, and single steps for the tail
-    with torch.cuda.stream(stream):
-        g_all = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g_all, stream=stream):
-            for i in range(copies):
-                step(i)
-        g_one = []
-        for i in range(copies):
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=stream):
-                step(i)
-            g_one.append(g)
-    torch.cuda.synchronize()
-
-    def run_steps(n):
-        full, rem = divmod(n, copies)
-        for _ in range(full):
-            g_all.replay()
-        for i in range(rem):
-            g_one[i].replay()
-
-    run_steps(max(3, args.warmup))
-    torch.cuda.synchronize()
-    if dist:
-        dist.barrier()
-    sampler = ClockSampler(local)
-    sampler.start()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    torch.cuda.synchronize()
-    if dist:
-        dist.barrier()
-    e0.record(stream)
-    run_steps(args.steps)
-    e1.record(stream)
-    e1.synchronize()
-    torch.cuda.synchronize()
-    if dist:
-        dist.barrier()
-    clocks = sampler.stop()
-    ms = e0.elapsed_time(e1)
-    if dist:
-        t = torch.tensor([ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-    if bl.bitlinear_get_status() != bl.BL_OK:
-        raise RuntimeError("device status word set during the timed region")
-
-    nbytes = block_bytes(lin, M)
-    value = nbytes * args.steps * world / (ms / 1e3) / 1e9
-    ms_step = ms / args.steps
-
-    # ---- dominant kernel: the product kernel (the whole step in grouped mode)
-    peak, peak_kind = load_peaks()
-    if args.mode == "grouped":
-        kern_ms, kern_bytes = ms_step, nbytes
+    if args.workload == "prefill":
+        sampler = ClockSampler(local)
+        sampler.start()
+        pf = run_prefill(torch, bl, args, dev, stream, dist, l2, max(8, args.steps // 100))
+        clocks = sampler.stop()
+        out = {"metric": METRIC, "value": pf["value"] * world, "unit": "TOPS", "n_gpus": world,
+               "steps": pf["steps"], "warmup": args.warmup, "ms_per_step": pf["ms_per_step"],
+               "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int32",
+               "data": "synthetic", "config": dict(config, l2_policy=pf["l2_policy"]),
+               "roofline": pf["roofline"], "gpu_launches": pf["launches_per_step"] * pf["steps"],
+               "clocks": clocks}
+        if rank == 0 and not args.no_cpu_baseline:
+            out["cpu_baseline"] = cpu_baseline(lin, args.cpu_seconds, prefill=True)
+    elif args.workload == "pack":
+        pk = run_pack(torch, bl, args, dev, stream, dist, l2)
+        out = {"metric": "absmean ternary quantise + 2-bit pack, GB/s", "value": pk["value"] * world,
+               "unit": "GB/s", "n_gpus": world, "steps": pk["steps"], "warmup": 3,
+               "ms_per_step": pk["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+               "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+               "config": {"workload": "pack_block2b", "note": pk["note"]},
+               "roofline": {"bound": "hbm", "achieved": pk["value"], "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                            "frac": pk["value"] / peaks["hbm_gbs"], "traffic": None},
+               "gpu_launches": pk["launches_per_step"] * pk["steps"]}
     else:
-        # time the product launches alone (no quantisation) over the same rotation
-        with torch.cuda.stream(stream):
-            gk = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(gk, stream=stream):
-                for i in range(copies):
-                    for j in range(len(lin)):
-                        if args.mode == "fused":
-                            bl.bitlinear_forward_x(xs[i][j], packed[i][j], g32s[j], Ns[j], Ks[j], ys[i][j], stream)
-                        else:
-                            bl.bitlinear_forward(qs[j], ss[j], packed[i][j], g32s[j], M, Ns[j], Ks[j], ys[i][j],
-                                                 None, stream)
-        reps = max(1, args.steps // copies)
-        gk.replay()
-        e0.record(stream)
-        for _ in range(reps):
-            gk.replay()
-        e1.record(stream)
-        e1.synchronize()
-        kern_ms = e0.elapsed_time(e1) / (reps * copies * len(lin))
-        kern_bytes = nbytes / len(lin)
-    achieved = kern_bytes / (kern_ms / 1e3) / 1e9
-    roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                "frac": achieved / peak, "traffic": None,
-                "kernel": "gemv_kernel (fused quant prologue, grouped over the 7 linears)"
-                if args.mode == "grouped" else "gemv_kernel",
-                "peak_kind": f"{peak_kind} HBM copy bandwidth (burst)",
-                "algorithmic_bytes_per_launch": kern_bytes, "avg_launch_us": kern_ms * 1e3}
-
-    # ---- end to end through the public API: pinned host x in, host y out
-    e2e = None
-    if not args.no_e2e:
-        hx = torch.empty(sum(M * K for K in Ks), dtype=torch.bfloat16).pin_memory()
-        hy = torch.empty(sum(M * N for N in Ns), dtype=torch.float32).pin_memory()
-        off = 0
-        for L in lin:
-            hx[off:off + M * L["K"]].copy_(torch.from_numpy(L["x"].view(np.int16).ravel()).view(torch.bfloat16))
-            off += M * L["K"]
-        dx = torch.empty_like(hx, device=dev)
-        dy = torch.empty_like(hy, device=dev)
-        xv, yv, ox, oy = [], [], 0, 0
-        for K, N in zip(Ks, Ns):
-            xv.append(dx[ox:ox + M * K].view(M, K))
-            yv.append(dy[oy:oy + M * N].view(M, N))
-            ox += M * K
-            oy += M * N
-        e2e_steps = max(1, min(args.steps, 2000))
-
-        def e2e_step(i):
-            c = i % copies
-            dx.copy_(hx, non_blocking=True)
-            bl.bitlinear_forward_x_grouped(xv, packed[c], g32s, Ns, Ks, yv, stream)
-            hy.copy_(dy, non_blocking=True)
-
-        for i in range(3):
-            e2e_step(i)
-        torch.cuda.synchronize()
-        e0.record(stream)
-        for i in range(e2e_steps):
-            e2e_step(i)
-        e1.record(stream)
-        e1.synchronize()
-        ems = e0.elapsed_time(e1)
-        if dist:
-            t = torch.tensor([ems], device=dev, dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ems = float(t.item())
-        e2e = {"value": nbytes * e2e_steps * world / (ems / 1e3) / 1e9, "unit": "GB/s",
-               "h2d_bytes_per_step": hx.numel() * hx.element_size(),
-               "d2h_bytes_per_step": hy.numel() * hy.element_size(),
-               "ms_per_step": ems / e2e_steps,
-               "path": "pinned host x -> H2D -> bitlinear_forward_x_grouped (C ABI) -> D2H y, per step"}
-
-    out = {"metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
-           "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-           "vs_baseline": None, "dtype": "int32", "data": "synthetic", "config": config,
-           "roofline": roofline, "e2e": e2e, "gpu_launches": launches_per_step * args.steps,
-           "clocks": clocks}
-    if rank == 0 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline(lin, args.cpu_seconds)
+        R = run_decode(torch, bl, args, lin, M, dev, stream, dist, l2)
+        nbytes, ms = R["nbytes"], R["ms"]
+        achieved = R["kern_bytes"] / (R["kern_ms"] / 1e3) / 1e9
+        config.update({"weight_copies": R["S"]["copies"], "rotating_bytes": R["S"]["per_copy"] * R["S"]["copies"],
+                       "l2_bytes": l2, "l2_policy": "inputs larger than L2: weights/x/y rotate over copies > 3x L2",
+                       "mode": R["mode"]})
+        out = {"metric": METRIC, "value": nbytes * args.steps * world / (ms / 1e3) / 1e9, "unit": "GB/s",
+               "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+               "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int32",
+               "data": "synthetic", "config": config,
+               "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                            "frac": achieved / peaks["hbm_gbs"], "traffic": None, "kernel": R["kname"],
+                            "peak_kind": f"{peaks['kind']} HBM copy bandwidth (burst)",
+                            "algorithmic_bytes_per_launch": R["kern_bytes"],
+                            "avg_launch_us": R["kern_ms"] * 1e3},
+               "gpu_launches": R["launches"] * args.steps, "clocks": R["clocks"]}
+        if not args.no_e2e and R["mode"] == "grouped":
+            ems, n, hb, db = run_e2e(torch, bl, lin, M, dev, stream, R["S"], args.steps, dist)
+            out["e2e"] = {"value": nbytes * n * world / (ems / 1e3) / 1e9, "unit": "GB/s",
+                          "h2d_bytes_per_step": hb, "d2h_bytes_per_step": db, "ms_per_step": ems / n,
+                          "path": "pinned host x -> H2D -> bitlinear_forward_x_grouped (C ABI) -> D2H y"}
+        if args.workload == "block2b" and not args.no_prefill:
+            out["prefill"] = run_prefill(torch, bl, args, dev, stream, dist, l2, 20)
+        if rank == 0 and not args.no_cpu_baseline:
+            out["cpu_baseline"] = cpu_baseline(lin, args.cpu_seconds)
     if dist:
         dist.barrier()
-        del g_all, g_one
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(out), flush=True)

@@ -112,9 +112,25 @@ bl_status bitlinear_forward(const int8_t* q, const float* s, const uint8_t* pack
     if (!status) return BL_ERR_CUDA;
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     if (M > bl::kFusedMaxM && bl::gemm_tc_supported(M, N, K))
-        return bl::launch_gemm_tc(q, s, packed, gamma32, M, N, K, y, yt, acc_debug, cs) == cudaSuccess
+        return bl::launch_gemm_tc(q, s, packed, gamma32, M, N, K, y, yt, acc_debug, status, cs) == cudaSuccess
                    ? BL_OK
                    : BL_ERR_CUDA;
+    if (M <= bl::kFusedMaxM) {
+        bl::StreamBatch sb;
+        std::memset(&sb, 0, sizeof(sb));
+        sb.count = 1;
+        sb.M = (int)M;
+        sb.p[0].q = q;
+        sb.p[0].s = s;
+        sb.p[0].packed = packed;
+        sb.p[0].gamma32 = gamma32;
+        sb.p[0].y = y;
+        sb.p[0].acc = acc_debug;
+        sb.p[0].N = N;
+        sb.p[0].K = K;
+        const cudaError_t e = bl::launch_stream(sb, false, BL_F32, yt, status, cs);
+        if (e != cudaErrorNotSupported) return e == cudaSuccess ? BL_OK : BL_ERR_CUDA;
+    }
     bl::GemvBatch b;
     std::memset(&b, 0, sizeof(b));
     b.count = 1;
@@ -162,9 +178,22 @@ bl_status bitlinear_forward_x_grouped(int count, const void* const* x, bl_dtype 
     if (tiles > (int64_t(1) << 31) - 1) return BL_ERR_SHAPE;
     unsigned* status = status_word();
     if (!status) return BL_ERR_CUDA;
-    return bl::launch_gemv(b, true, xt, yt, status, static_cast<cudaStream_t>(stream)) == cudaSuccess
-               ? BL_OK
-               : BL_ERR_CUDA;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    bl::StreamBatch sb;
+    std::memset(&sb, 0, sizeof(sb));
+    sb.count = count;
+    sb.M = (int)M;
+    for (int i = 0; i < count; ++i) {
+        sb.p[i].x = x[i];
+        sb.p[i].packed = packed[i];
+        sb.p[i].gamma32 = gamma32[i];
+        sb.p[i].y = y[i];
+        sb.p[i].N = N[i];
+        sb.p[i].K = K[i];
+    }
+    const cudaError_t e = bl::launch_stream(sb, true, xt, yt, status, cs);
+    if (e != cudaErrorNotSupported) return e == cudaSuccess ? BL_OK : BL_ERR_CUDA;
+    return bl::launch_gemv(b, true, xt, yt, status, cs) == cudaSuccess ? BL_OK : BL_ERR_CUDA;
 }
 
 bl_status bitlinear_forward_x(const void* x, bl_dtype xt, const uint8_t* packed, const float* gamma32,

@@ -1,14 +1,347 @@
-// bl_gemm_tc.cu -- prefill tensor-core path (tcgen05 kind::i8); see below.
+// bl_gemm_tc.cu -- prefill BitLinear on the 5th-generation tensor cores
+// (tcgen05 kind::i8): D[n, m] = sum_k code[n, k] * q[m, k] with int32
+// accumulation in tensor memory, then y[m, n] = D * (gamma32 / s_m).
+// (bhfrc.com/news/56965 sec. 1.1: ternary weights make the product pure
+// integer adds; aratech.ae "BitLinear: the building block" for the int8
+// per-token activations.)
+//
+// Tile: 128 weight rows (MMA M) x 256 tokens (MMA N) per CTA, K in stages of
+// 128.  The weights never exist as int8 in memory: the packed 2-bit codes
+// are TMA-loaded (4 KiB per stage), four expansion warps decode them to
+// signed int8 in registers and write them straight into tensor memory with
+// tcgen05.st, where the MMA reads them as its A operand.  Shared memory only
+// carries the activation tiles (B operand, TMA with 128-byte swizzle).
+//
+// Warp roles (256 threads):
+//   warp 0      TMEM allocation; TMA producer (one lane)
+//   warp 1      MMA issuer (one lane): 4 x tcgen05.mma (K = 32) per stage,
+//               tcgen05.commit -> stage-free barrier, final commit -> accum
+//   warps 2-3   per-token rescale factors gamma32 / s_m (fp64)
+//   warps 4-7   expansion (TMEM lanes 32*(w-4) ..), then the epilogue:
+//               tcgen05.ld of the accumulator, rescale, store y
+// All mbarrier waits are bounded (bl_ptx.cuh).
+//
+// Decode to signed int8: per 2-bit field (lo, hi), code = lo - hi.
+//   S = (w & 0x55555555 | 0xAAAAAAAA) - ((w >> 1) & 0x55555555)
+// holds 2 + code in every field (no borrow between fields; padding 11 -> 2,
+// i.e. code 0).  Field t of every byte, ((S >> 2t) & 0x03030303), plus
+// 0x7E7E7E7E then xor 0x80808080 gives the bytes 0xFF, 0x00, 0x01.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include "bl_internal.cuh"
+#include "bl_ptx.cuh"
 
 namespace bl {
+namespace {
 
-bool gemm_tc_supported(int64_t, int64_t, int64_t) { return false; }
+constexpr int BM = 128;        // weight rows per tile (MMA M)
+constexpr int BN = 256;        // tokens per tile (MMA N)
+constexpr int BK = 128;        // k per stage (bytes of int8)
+constexpr int STAGES = 4;
+constexpr int kThreads = 256;
+constexpr int Q_STAGE = BN * BK;             // 32 KiB, 128B-swizzled
+constexpr int W_STAGE = (BM / 8) * 256;      // 16 tiles x 2 chunks x 128 B = 4 KiB
+constexpr int TMEM_COLS = 512;
+constexpr int A_COL0 = 256;                  // A stages after the accumulator
+constexpr int A_STAGE_COLS = BK / 4;         // 32 columns per stage
 
-cudaError_t launch_gemm_tc(const int8_t*, const float*, const uint8_t*, const float*, int64_t, int64_t,
-                           int64_t, void*, bl_dtype, int32_t*, cudaStream_t)
+struct Smem {
+    uint8_t q[STAGES][Q_STAGE];              // 1024-aligned (first member)
+    uint8_t w[STAGES][W_STAGE];
+    double fac[BN];
+    uint64_t full[STAGES], expanded[STAGES], empty[STAGES], accum;
+    uint32_t tmem_base;
+    int abort_flag;
+};
+
+__device__ __forceinline__ uint32_t signed_codes(int t, uint32_t S)
 {
-    return cudaErrorNotSupported;
+    return (((S >> (2 * t)) & 0x03030303u) + 0x7E7E7E7Eu) ^ 0x80808080u;
+}
+
+__device__ __forceinline__ uint64_t make_bdesc(uint32_t smem_addr)
+{
+    // K-major, 128-byte swizzle: rows of 128 B, 8-row core groups 1024 B apart.
+    uint64_t d = 0;
+    d |= (uint64_t)((smem_addr >> 4) & 0x3FFF);          // start address
+    d |= (uint64_t)1 << 16;                               // leading byte offset (unused for SW128 K-major)
+    d |= (uint64_t)(1024 >> 4) << 32;                     // stride byte offset
+    d |= (uint64_t)1 << 46;                               // descriptor version (sm_100)
+    d |= (uint64_t)2 << 61;                               // SWIZZLE_128B
+    return d;
+}
+
+// kind::i8, D = S32, A = B = signed int8, both K-major, M = 128, N = 256.
+constexpr uint32_t kIdesc = (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
+                            ((uint32_t)(BM >> 4) << 24);
+
+__device__ __forceinline__ void mma_i8_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(kIdesc), "r"(accumulate)
+        : "memory");
+}
+
+__device__ __forceinline__ void mma_commit(uint64_t* bar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     smem_u32(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32])
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, "
+        "%13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(
+            taddr),
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
+        "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]),
+        "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]),
+        "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32])
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+        "%14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+          "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]),
+          "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]),
+          "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]),
+          "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+        : "r"(taddr)
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ void store_y(float* y, int64_t i, float v) { y[i] = v; }
+__device__ __forceinline__ void store_y(__nv_bfloat16* y, int64_t i, float v) { y[i] = __float2bfloat16_rn(v); }
+
+template <typename YT>
+__global__ void __launch_bounds__(kThreads, 1)
+gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_w,
+               const float* __restrict__ s_in, const float* __restrict__ gamma32, int M, int N, int nk,
+               YT* __restrict__ y, int32_t* __restrict__ acc_out, unsigned* status)
+{
+    extern __shared__ uint8_t smem_raw[];
+    Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n0 = blockIdx.x * BM, m0 = blockIdx.y * BN;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&sm.full[s], 1);
+            mbar_init(&sm.expanded[s], 128);
+            mbar_init(&sm.empty[s], 1);
+        }
+        mbar_init(&sm.accum, 1);
+        sm.abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0) {
+        __syncwarp();
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(&sm.tmem_base)),
+                     "r"(TMEM_COLS)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+    volatile int* abort = &sm.abort_flag;
+
+    if (warp == 0) {
+        // ---------------------------------------------------- TMA producer
+        if (lane == 0) {
+            prefetch_tmap(&tmap_q);
+            prefetch_tmap(&tmap_w);
+            int issued = 0;
+            for (int kb = 0; kb < nk; ++kb) {
+                const int s = kb % STAGES, round = kb / STAGES;
+                if (round > 0 && !wait_parity(&sm.empty[s], (round - 1) & 1, status, abort)) break;
+                mbar_arrive_expect_tx(&sm.full[s], Q_STAGE + W_STAGE);
+                tma_load_2d(sm.q[s], &tmap_q, kb * BK, m0, &sm.full[s]);
+                tma_load_2d(sm.w[s], &tmap_w, kb * 256, n0 / 8, &sm.full[s]);
+                issued = kb + 1;
+            }
+            for (int kb = issued - STAGES < 0 ? 0 : issued - STAGES; kb < issued; ++kb)
+                wait_parity(&sm.full[kb % STAGES], (kb / STAGES) & 1, status, nullptr);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            for (int kb = 0; kb < nk; ++kb) {
+                const int s = kb % STAGES;
+                const uint32_t ph = (kb / STAGES) & 1;
+                if (!wait_parity(&sm.full[s], ph, status, abort)) break;
+                if (!wait_parity(&sm.expanded[s], ph, status, abort)) break;
+                tc_fence_after();
+                const uint32_t qaddr = smem_u32(sm.q[s]);
+#pragma unroll
+                for (int j = 0; j < BK / 32; ++j)
+                    mma_i8_ts(tmem, tmem + A_COL0 + s * A_STAGE_COLS + j * 8, make_bdesc(qaddr + j * 32),
+                              (kb | j) != 0);
+                mma_commit(&sm.empty[s]);
+            }
+            mma_commit(&sm.accum);   // also on abort: retires every MMA issued
+        }
+    } else if (warp < 4) {
+        // -------------------------------------------------- rescale factors
+        const double g = (double)*gamma32;
+        for (int j = threadIdx.x - 64; j < BN; j += 64) {
+            const int m = m0 + j;
+            sm.fac[j] = (m < M) ? g / (double)s_in[m] : 0.0;
+        }
+    } else {
+        // --------------------------------------------- expansion warps 4..7
+        const int rr = threadIdx.x - 128;          // TMEM lane = weight row in tile
+        const int quarter = warp - 4;
+        const uint32_t lane_base = (uint32_t)(32 * quarter) << 16;
+        const int woff = (rr >> 3) * 256 + (rr & 7) * 16;
+        for (int kb = 0; kb < nk; ++kb) {
+            const int s = kb % STAGES;
+            const bool got = wait_parity(&sm.full[s], (kb / STAGES) & 1, status, abort);
+            if (!__all_sync(0xffffffffu, got)) break;   // warp-uniform: tcgen05.st is .aligned
+            uint32_t out[32];
+#pragma unroll
+            for (int cl = 0; cl < 2; ++cl) {
+                const uint4 wv = *reinterpret_cast<const uint4*>(sm.w[s] + woff + cl * 128);
+                const uint32_t words[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const uint32_t w = words[i];
+                    const uint32_t S = ((w & 0x55555555u) | 0xAAAAAAAAu) - ((w >> 1) & 0x55555555u);
+#pragma unroll
+                    for (int t = 0; t < 4; ++t) out[16 * cl + 4 * i + t] = signed_codes(t, S);
+                }
+            }
+            tmem_st32(tmem + lane_base + A_COL0 + s * A_STAGE_COLS, out);
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(&sm.expanded[s]);
+        }
+        // ------------------------------------------------------- epilogue
+        __syncwarp();
+        named_bar(2, 128 + 64);   // factors ready (warps 2-7)
+        const bool ok = __all_sync(0xffffffffu, wait_parity(&sm.accum, 0, status, abort));
+        tc_fence_after();
+        const int n = n0 + rr;
+        if (ok) {
+#pragma unroll 1
+            for (int cc = 0; cc < BN / 32; ++cc) {
+                uint32_t v[32];
+                tmem_ld32(tmem + lane_base + cc * 32, v);
+                tmem_wait_ld();
+                if (n < N) {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const int m = m0 + cc * 32 + j;
+                        if (m < M) {
+                            const int a = (int)v[j];
+                            const int64_t o = (int64_t)m * N + n;
+                            if (acc_out) acc_out[o] = a;
+                            store_y(y, o, (float)((double)a * sm.fac[cc * 32 + j]));
+                        }
+                    }
+                }
+            }
+        }
+        tc_fence_before();
+    }
+    if (warp == 2 || warp == 3) named_bar(2, 128 + 64);
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS)
+                     : "memory");
+    }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult qr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &qr) == cudaSuccess &&
+            qr == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+bool make_2d_u8(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint64_t stride,
+                uint32_t box_in, uint32_t box_out, CUtensorMapSwizzle sw)
+{
+    auto fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {inner, outer};
+    const cuuint64_t strides[1] = {stride};
+    const cuuint32_t box[2] = {box_in, box_out};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <typename YT>
+cudaError_t launch_typed(const CUtensorMap& tq, const CUtensorMap& tw, const float* s, const float* g, int M,
+                         int N, int nk, void* y, int32_t* acc, unsigned* status, cudaStream_t st)
+{
+    const size_t smem = sizeof(Smem) + 1024;
+    static bool configured[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!configured[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<YT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)smem);
+        if (e != cudaSuccess) return e;
+        configured[dev] = true;
+    }
+    dim3 grid((N + BM - 1) / BM, (M + BN - 1) / BN);
+    gemm_tc_kernel<YT><<<grid, kThreads, smem, st>>>(tq, tw, s, g, M, N, nk, static_cast<YT*>(y), acc, status);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool gemm_tc_supported(int64_t M, int64_t N, int64_t K)
+{
+    return M > 16 && M < (int64_t(1) << 31) && N < (int64_t(1) << 31) && (M + BN - 1) / BN <= 65535 &&
+           padded_k(K) < (int64_t(1) << 31) && encode_fn() != nullptr;
+}
+
+cudaError_t launch_gemm_tc(const int8_t* q, const float* s, const uint8_t* packed, const float* gamma32,
+                           int64_t M, int64_t N, int64_t K, void* y, bl_dtype yt, int32_t* acc,
+                           unsigned* status, cudaStream_t st)
+{
+    const int64_t Kp = padded_k(K);
+    const int64_t TB = chunks_per_row(K) * 128;
+    CUtensorMap tq, tw;
+    if (!make_2d_u8(&tq, q, (uint64_t)Kp, (uint64_t)M, (uint64_t)Kp, BK, BN, CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    if (!make_2d_u8(&tw, packed, (uint64_t)TB, (uint64_t)(padded_n(N) / 8), (uint64_t)TB, 256, BM / 8,
+                    CU_TENSOR_MAP_SWIZZLE_NONE))
+        return cudaErrorInvalidValue;
+    const int nk = (int)((Kp + BK - 1) / BK);
+    if (yt == BL_F32)
+        return launch_typed<float>(tq, tw, s, gamma32, (int)M, (int)N, nk, y, acc, status, st);
+    return launch_typed<__nv_bfloat16>(tq, tw, s, gamma32, (int)M, (int)N, nk, y, acc, status, st);
 }
 
 }  // namespace bl

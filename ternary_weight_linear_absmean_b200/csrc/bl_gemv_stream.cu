@@ -1,0 +1,492 @@
+// bl_gemv_stream.cu -- persistent, HBM-streaming decode kernel (M <= 16):
+// packed ternary weights x int8 activations -> int32 -> y = acc * gamma / s
+// (bhfrc.com/news/56965 sec. 1.1: a ternary weight adds, subtracts or skips
+// an activation; aratech.ae "BitLinear: the building block" for the int8
+// per-token activations).
+//
+// Launch: two CTAs per SM.  CTAs are shared out among the problems of the
+// launch in proportion to their packed bytes, and each CTA owns a contiguous
+// range of whole 8-row tiles of one problem -- in the packed layout that is
+// one contiguous byte range.
+//
+// Inside a CTA (8 warps):
+//   warp 0, lane 0  producer: streams the range into a ring of 16 KiB shared
+//                   memory stages with 1-D bulk copies (cp.async.bulk), one
+//                   mbarrier pair (full/empty) per stage;
+//   warps 1..7      consumers: first quantise x into shared memory (fused
+//                   form) or copy q there, while the first stages are in
+//                   flight; then for each stage take 512-byte spans (4 chunks
+//                   x 8 rows of a tile) round-robin, lane l reading 16 bytes,
+//                   row r = l % 8, and accumulate with dp4a (decode as in
+//                   bl_gemv.cu).  Per-lane partial sums are added into a
+//                   per-(tile, row, token) int32 array in shared memory
+//                   (integer adds: exact and order-independent) whenever the
+//                   lane's tile changes.
+//   epilogue        y = (float)((double)acc * (double)gamma32 / (double)s_m),
+//                   bit-identical to the oracle's rescale.
+#include "bl_internal.cuh"
+#include "bl_ptx.cuh"
+
+namespace bl {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kConsumerWarps = 7;
+constexpr int kConsumers = kConsumerWarps * 32;
+constexpr int kStageBytes = 16384;
+constexpr int kSpan = 512;
+
+__device__ __forceinline__ float to_f(float v) { return v; }
+__device__ __forceinline__ float to_f(__nv_bfloat16 v) { return __bfloat162float(v); }
+__device__ __forceinline__ void store_y(float* y, int64_t i, float v) { y[i] = v; }
+__device__ __forceinline__ void store_y(__nv_bfloat16* y, int64_t i, float v) { y[i] = __float2bfloat16_rn(v); }
+
+__device__ __forceinline__ int8_t quant_one(float v, float s)
+{
+    float r = rintf(__fmul_rn(v, s));
+    r = fminf(fmaxf(r, -127.0f), 127.0f);
+    return (int8_t)(int)r;
+}
+
+// max over the 224 consumer threads (named barrier 1)
+__device__ __forceinline__ float consumers_max(float v, float* red)
+{
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    const int cw = (threadIdx.x >> 5) - 1;
+    if ((threadIdx.x & 31) == 0) red[cw] = v;
+    named_bar(1, kConsumers);
+    float m = red[0];
+#pragma unroll
+    for (int w = 1; w < kConsumerWarps; ++w) m = fmaxf(m, red[w]);
+    return m;
+}
+
+__device__ __forceinline__ int consumers_sum(int v, int* red)
+{
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    const int cw = (threadIdx.x >> 5) - 1;
+    if ((threadIdx.x & 31) == 0) red[cw] = v;
+    named_bar(1, kConsumers);
+    int t = 0;
+#pragma unroll
+    for (int w = 0; w < kConsumerWarps; ++w) t += red[w];
+    return t;
+}
+
+// Quantise x row (K elements) into q (Kp bytes) in shared memory; returns s.
+// Same arithmetic as bl_quant.cu: amax over the row, s = 127 / max(amax,
+// 1e-5) (IEEE divide), q = clamp(rint(x * s), -127, 127) in fp32.
+template <typename XT>
+__device__ float quantise_row(const XT* __restrict__ row, int K, int Kp, int8_t* q, float* redf, int* redi,
+                              int* sumq_out, unsigned* status)
+{
+    const int t = threadIdx.x - 32;
+    constexpr int VE = 16 / sizeof(XT);   // elements per 16-byte vector
+    const bool vec = (K % VE) == 0;
+    float amax = 0.0f;
+    bool bad = false;
+    if (vec) {
+        const uint4* rv = reinterpret_cast<const uint4*>(row);
+        for (int v = t; v < K / VE; v += kConsumers) {
+            const uint4 u = __ldg(rv + v);
+            const XT* e = reinterpret_cast<const XT*>(&u);
+#pragma unroll
+            for (int i = 0; i < VE; ++i) {
+                const float f = to_f(e[i]);
+                bad |= !isfinite(f);
+                amax = fmaxf(amax, fabsf(f));
+            }
+        }
+    } else {
+        for (int k = t; k < K; k += kConsumers) {
+            const float f = to_f(row[k]);
+            bad |= !isfinite(f);
+            amax = fmaxf(amax, fabsf(f));
+        }
+    }
+    if (bad) atomicOr(status, kStatusNonfiniteX);
+    amax = fmaxf(consumers_max(amax, redf), 1e-5f);
+    const float s = 127.0f / amax;
+    int part = 0;
+    if (vec) {
+        const uint4* rv = reinterpret_cast<const uint4*>(row);
+        for (int v = t; v < K / VE; v += kConsumers) {
+            const uint4 u = __ldg(rv + v);
+            const XT* e = reinterpret_cast<const XT*>(&u);
+            uint32_t words[VE / 4];
+#pragma unroll
+            for (int w = 0; w < VE / 4; ++w) {
+                uint32_t word = 0;
+#pragma unroll
+                for (int b = 0; b < 4; ++b) word |= (uint32_t)(uint8_t)quant_one(to_f(e[4 * w + b]), s) << (8 * b);
+                words[w] = word;
+                part = dp4a_ss(word, 0x01010101u, part);
+            }
+            if constexpr (VE == 8)
+                *reinterpret_cast<uint2*>(q + v * 8) = make_uint2(words[0], words[1]);
+            else
+                *reinterpret_cast<uint32_t*>(q + v * 4) = words[0];
+        }
+        for (int k4 = K + 4 * t; k4 < Kp; k4 += 4 * kConsumers) *reinterpret_cast<uint32_t*>(q + k4) = 0u;
+    } else {
+        for (int k4 = 4 * t; k4 < Kp; k4 += 4 * kConsumers) {
+            uint32_t word = 0;
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+                const int k = k4 + b;
+                const int8_t v = (k < K) ? quant_one(to_f(row[k]), s) : (int8_t)0;
+                word |= (uint32_t)(uint8_t)v << (8 * b);
+            }
+            *reinterpret_cast<uint32_t*>(q + k4) = word;
+            part = dp4a_ss(word, 0x01010101u, part);
+        }
+    }
+    *sumq_out = consumers_sum(part, redi);
+    return s;
+}
+
+template <int MT>
+__device__ __forceinline__ void dot_chunk(const uint4 wv, const int8_t* qs, int Kp, int c, int M, int (&acc)[MT][4])
+{
+    const uint32_t U[4] = {biased_codes(wv.x), biased_codes(wv.y), biased_codes(wv.z), biased_codes(wv.w)};
+#pragma unroll
+    for (int m = 0; m < MT; ++m) {
+        if (m < M) {
+            const uint4* a4 = reinterpret_cast<const uint4*>(qs + m * Kp + c * 64);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const uint4 a = a4[i];
+                acc[m][0] = dp4a_us(U[i] & 0x03030303u, a.x, acc[m][0]);
+                acc[m][1] = dp4a_us(U[i] & 0x0C0C0C0Cu, a.y, acc[m][1]);
+                acc[m][2] = dp4a_us(U[i] & 0x30303030u, a.z, acc[m][2]);
+                acc[m][3] = dp4a_us(U[i] & 0xC0C0C0C0u, a.w, acc[m][3]);
+            }
+        }
+    }
+}
+
+template <int MT, bool FUSED, typename XT, typename YT, int MINB>
+__global__ void __launch_bounds__(kThreads, MINB)
+stream_kernel(const __grid_constant__ StreamBatch b, unsigned* status)
+{
+    extern __shared__ __align__(128) uint8_t smem[];
+    __shared__ uint64_t full_bar[kMaxStages], empty_bar[kMaxStages];
+    __shared__ float s_scale[MT];
+    __shared__ int s_sumq[MT];
+    __shared__ float redf[kConsumerWarps];
+    __shared__ int redi[kConsumerWarps];
+    __shared__ int abort_flag;
+
+    // ---- which problem, which tiles
+    int pi = 0;
+#pragma unroll 1
+    for (int i = 1; i < b.count; ++i)
+        if ((int)blockIdx.x >= b.p[i].cta_begin) pi = i;
+    const StreamProblem& P = b.p[pi];
+    const int K = (int)P.K, Kp = (int)padded_k(P.K);
+    const int64_t N = P.N;
+    const uint32_t TB = (uint32_t)(chunks_per_row(K) * 128);   // bytes per tile
+    const int64_t tiles = padded_n(N) / 8;
+    const int64_t ci = (int64_t)blockIdx.x - P.cta_begin;
+    const int64_t t0 = tiles * ci / P.ctas, t1 = tiles * (ci + 1) / P.ctas;
+    const uint32_t range = (uint32_t)((t1 - t0) * TB);            // < 2^31 (host-checked)
+    const uint8_t* src = P.packed + t0 * (int64_t)TB;
+    const int stages = b.stages;
+    const int npieces = (int)((range + kStageBytes - 1) / kStageBytes);
+
+    uint8_t* ring = smem;
+    int8_t* qs = reinterpret_cast<int8_t*>(smem + (size_t)stages * kStageBytes);
+    int* sacc = reinterpret_cast<int*>(smem + (size_t)stages * kStageBytes + b.q_bytes);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < stages; ++s) {
+            mbar_init(&full_bar[s], 1);
+            mbar_init(&empty_bar[s], kConsumerWarps);
+        }
+        abort_flag = 0;
+        fence_barrier_init();
+    }
+    __syncthreads();
+
+    if (warp == 0) {
+        // ------------------------------------------------------ producer
+        if (lane == 0) {
+            int issued = 0;
+            for (int j = 0; j < npieces; ++j) {
+                const int s = j % stages, round = j / stages;
+                if (round > 0 && !wait_parity(&empty_bar[s], (round - 1) & 1, status, &abort_flag)) break;
+                const uint32_t left = range - (uint32_t)j * kStageBytes;
+                const uint32_t len = left < (uint32_t)kStageBytes ? left : (uint32_t)kStageBytes;
+                mbar_arrive_expect_tx(&full_bar[s], len);
+                bulk_g2s(ring + (size_t)s * kStageBytes, src + (int64_t)j * kStageBytes, len, &full_bar[s]);
+                issued = j + 1;
+            }
+            // every copy this thread issued lands before it exits (the last
+            // use of each stage is that stage's latest phase)
+            for (int j = issued - stages < 0 ? 0 : issued - stages; j < issued; ++j)
+                wait_parity(&full_bar[j % stages], (j / stages) & 1, status, nullptr);
+        }
+        return;
+    }
+
+    // ---------------------------------------------------------- consumers
+    const int cw = warp - 1;
+    const int M = b.M;
+    const int ntl = (int)(t1 - t0);
+    for (int i = threadIdx.x - 32; i < ntl * 8 * MT; i += kConsumers) sacc[i] = 0;
+    if constexpr (FUSED) {
+        const XT* xb = static_cast<const XT*>(P.x);
+#pragma unroll 1
+        for (int m = 0; m < M; ++m) {
+            int sq;
+            const float s = quantise_row<XT>(xb + (int64_t)m * K, K, Kp, qs + m * Kp, redf, redi, &sq, status);
+            if (threadIdx.x == 32) {
+                s_scale[m] = s;
+                s_sumq[m] = sq;
+            }
+            named_bar(1, kConsumers);
+        }
+    } else {
+#pragma unroll 1
+        for (int m = 0; m < M; ++m) {
+            const uint4* gq = reinterpret_cast<const uint4*>(P.q + (int64_t)m * Kp);
+            uint4* sq4 = reinterpret_cast<uint4*>(qs + m * Kp);
+            int part = 0;
+            for (int v = threadIdx.x - 32; v < Kp / 16; v += kConsumers) {
+                const uint4 u = __ldg(gq + v);
+                sq4[v] = u;
+                part = dp4a_ss(u.x, 0x01010101u, part);
+                part = dp4a_ss(u.y, 0x01010101u, part);
+                part = dp4a_ss(u.z, 0x01010101u, part);
+                part = dp4a_ss(u.w, 0x01010101u, part);
+            }
+            const int sq = consumers_sum(part, redi);
+            if (threadIdx.x == 32) {
+                s_scale[m] = P.s[m];
+                s_sumq[m] = sq;
+            }
+            named_bar(1, kConsumers);
+        }
+    }
+
+    const int r = lane & 7;
+    int cur = -1;
+    int acc[MT][4];
+#pragma unroll
+    for (int m = 0; m < MT; ++m)
+#pragma unroll
+        for (int t = 0; t < 4; ++t) acc[m][t] = 0;
+
+    auto flush = [&]() {
+        if (cur >= 0) {
+#pragma unroll
+            for (int m = 0; m < MT; ++m) {
+                if (m < M) {
+                    const int tot = acc[m][0] + (acc[m][1] >> 2) + (acc[m][2] >> 4) + (acc[m][3] >> 6);
+                    atomicAdd(&sacc[(cur * 8 + r) * MT + m], tot);
+                }
+#pragma unroll
+                for (int t = 0; t < 4; ++t) acc[m][t] = 0;
+            }
+        }
+    };
+
+    constexpr uint32_t kStep = kConsumerWarps * kSpan;   // bytes between a warp's spans
+#pragma unroll 1
+    for (int j = 0; j < npieces; ++j) {
+        const int s = j % stages, round = j / stages;
+        if (!wait_parity(&full_bar[s], round & 1, status, &abort_flag)) break;
+        const uint32_t poff = (uint32_t)j * kStageBytes;
+        const uint32_t len = (range - poff) < (uint32_t)kStageBytes ? (range - poff) : (uint32_t)kStageBytes;
+        const uint8_t* stage = ring + (size_t)s * kStageBytes;
+        // lane's position: one division per stage, then incremental
+        uint32_t boff = (uint32_t)cw * kSpan + (uint32_t)lane * 16;
+        uint32_t tile = (poff + boff) / TB;
+        uint32_t within = (poff + boff) - tile * TB;
+        uint4 wnext = make_uint4(0, 0, 0, 0);
+        if (boff < len) wnext = *reinterpret_cast<const uint4*>(stage + boff);
+#pragma unroll 1
+        for (uint32_t sb = (uint32_t)cw * kSpan; sb < len; sb += kStep, boff += kStep) {
+            const uint4 wv = wnext;
+            if (boff + kStep < len) wnext = *reinterpret_cast<const uint4*>(stage + boff + kStep);
+            if (boff < len) {
+                if ((int)tile != cur) {
+                    flush();
+                    cur = (int)tile;
+                }
+                dot_chunk<MT>(wv, qs, Kp, (int)(within >> 7), M, acc);
+            }
+            within += kStep;
+            if (within >= TB) {
+                if (TB >= kStep) {
+                    within -= TB;
+                    ++tile;
+                } else {
+                    tile += within / TB;
+                    within %= TB;
+                }
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty_bar[s]);
+    }
+    flush();
+    named_bar(1, kConsumers);
+    if (abort_flag) return;
+
+    // ---------------------------------------------------------- epilogue
+    const float g32 = *P.gamma32;
+    for (int i = threadIdx.x - 32; i < ntl * 8 * M; i += kConsumers) {
+        const int m = i % M;
+        const int row = i / M;                    // tile_local * 8 + r
+        const int64_t n = t0 * 8 + row;
+        if (n < N) {
+            const int a = sacc[row * MT + m] - s_sumq[m];
+            const int64_t o = (int64_t)m * N + n;
+            if (P.acc) P.acc[o] = a;
+            store_y(static_cast<YT*>(P.y), o, (float)((double)a * (double)g32 / (double)s_scale[m]));
+        }
+    }
+}
+
+template <int MT, bool FUSED, typename XT, typename YT, int MINB>
+cudaError_t launch_t(const StreamBatch& b, int grid, size_t smem, unsigned* status, cudaStream_t st)
+{
+    auto fn = stream_kernel<MT, FUSED, XT, YT, MINB>;
+    static bool configured[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!configured[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, stream_budget(MINB));
+        if (e != cudaSuccess) return e;
+        configured[dev] = true;
+    }
+    fn<<<grid, kThreads, smem, st>>>(b, status);
+    return cudaGetLastError();
+}
+
+template <bool FUSED, typename XT, typename YT, int MINB>
+cudaError_t launch_m(const StreamBatch& b, int grid, size_t smem, unsigned* status, cudaStream_t st)
+{
+    switch (stream_tokens(b.M)) {
+        case 1: return launch_t<1, FUSED, XT, YT, MINB>(b, grid, smem, status, st);
+        case 2: return launch_t<2, FUSED, XT, YT, MINB>(b, grid, smem, status, st);
+        case 4: return launch_t<4, FUSED, XT, YT, MINB>(b, grid, smem, status, st);
+        case 8: return launch_t<8, FUSED, XT, YT, MINB>(b, grid, smem, status, st);
+        default: return launch_t<16, FUSED, XT, YT, MINB>(b, grid, smem, status, st);
+    }
+}
+
+// 4 CTAs per SM (64 registers) only for up to 4 tokens; more tokens need
+// the registers of the 2-CTA form.
+template <bool FUSED, typename XT, typename YT>
+cudaError_t launch_b(const StreamBatch& b, int minb, int grid, size_t smem, unsigned* status, cudaStream_t st)
+{
+    if (minb == 4) {
+        switch (stream_tokens(b.M)) {
+            case 1: return launch_t<1, FUSED, XT, YT, 4>(b, grid, smem, status, st);
+            case 2: return launch_t<2, FUSED, XT, YT, 4>(b, grid, smem, status, st);
+            case 4: return launch_t<4, FUSED, XT, YT, 4>(b, grid, smem, status, st);
+            default: return cudaErrorNotSupported;
+        }
+    }
+    return launch_m<FUSED, XT, YT, 2>(b, grid, smem, status, st);
+}
+
+}  // namespace
+
+int stream_tokens(int64_t M) { return M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : M <= 8 ? 8 : 16; }
+
+int sm_count()
+{
+    static int cached[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (!cached[dev]) {
+        int v = 0;
+        if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 148;
+        cached[dev] = v;
+    }
+    return cached[dev];
+}
+
+// Plans CTAs per problem (proportional to packed bytes) and the shared
+// memory split for `minb` resident CTAs per SM.  Returns false if the
+// problems do not fit.
+bool plan_stream(StreamBatch& b, int minb, int* grid, size_t* smem)
+{
+    const int target = minb * sm_count();
+    const int MT = stream_tokens(b.M);
+    int64_t total = 0, kp_max = 0;
+    for (int i = 0; i < b.count; ++i) {
+        const int64_t bytes = padded_n(b.p[i].N) * padded_k(b.p[i].K) / 4;
+        if (bytes >= (int64_t(1) << 31)) return false;
+        total += bytes;
+        kp_max = kp_max > padded_k(b.p[i].K) ? kp_max : padded_k(b.p[i].K);
+    }
+    // CTAs per problem: largest-remainder share of `target`, >= 1, <= tiles
+    int assigned = 0;
+    double rem[kMaxGroup];
+    for (int i = 0; i < b.count; ++i) {
+        const int64_t bytes = padded_n(b.p[i].N) * padded_k(b.p[i].K) / 4;
+        const double share = (double)target * (double)bytes / (double)total;
+        int c = (int)share;
+        if (c < 1) c = 1;
+        b.p[i].ctas = c;
+        rem[i] = share - c;
+        assigned += c;
+    }
+    while (assigned < target) {
+        int best = 0;
+        for (int i = 1; i < b.count; ++i)
+            if (rem[i] > rem[best]) best = i;
+        b.p[best].ctas++;
+        rem[best] -= 1.0;
+        assigned++;
+    }
+    int64_t tiles_max = 1;
+    int begin = 0;
+    for (int i = 0; i < b.count; ++i) {
+        const int64_t tiles = padded_n(b.p[i].N) / 8;
+        if (b.p[i].ctas > tiles) b.p[i].ctas = (int)tiles;
+        b.p[i].cta_begin = begin;
+        begin += b.p[i].ctas;
+        const int64_t per = (tiles + b.p[i].ctas - 1) / b.p[i].ctas;
+        tiles_max = tiles_max > per ? tiles_max : per;
+    }
+    b.q_bytes = (int)(MT * kp_max);
+    const int64_t acc_bytes = tiles_max * 8 * MT * 4;
+    const int64_t left = (int64_t)stream_budget(minb) - b.q_bytes - acc_bytes;
+    int stages = (int)(left / 16384);
+    if (stages > kMaxStages) stages = kMaxStages;
+    if (stages < 2) return false;
+    b.stages = stages;
+    *grid = begin;
+    *smem = (size_t)stages * 16384 + b.q_bytes + acc_bytes;
+    return true;
+}
+
+cudaError_t launch_stream(StreamBatch& b, bool fused, bl_dtype xt, bl_dtype yt, unsigned* status,
+                          cudaStream_t st)
+{
+    int grid = 0, minb = stream_tokens(b.M) <= 4 ? 4 : 2;
+    size_t smem = 0;
+    if (!plan_stream(b, minb, &grid, &smem)) {
+        minb = 2;
+        if (!plan_stream(b, minb, &grid, &smem)) return cudaErrorNotSupported;
+    }
+    if (!fused) {
+        if (yt == BL_F32) return launch_b<false, float, float>(b, minb, grid, smem, status, st);
+        return launch_b<false, float, __nv_bfloat16>(b, minb, grid, smem, status, st);
+    }
+    if (xt == BL_F32) {
+        if (yt == BL_F32) return launch_b<true, float, float>(b, minb, grid, smem, status, st);
+        return launch_b<true, float, __nv_bfloat16>(b, minb, grid, smem, status, st);
+    }
+    if (yt == BL_F32) return launch_b<true, __nv_bfloat16, float>(b, minb, grid, smem, status, st);
+    return launch_b<true, __nv_bfloat16, __nv_bfloat16>(b, minb, grid, smem, status, st);
+}
+
+}  // namespace bl

@@ -65,12 +65,42 @@ cudaError_t launch_gemv(const GemvBatch& b, bool fused, bl_dtype xt, bl_dtype yt
 // Largest M the fused decode kernel accepts.
 constexpr int kFusedMaxM = 16;
 
+// Persistent streaming decode kernel (bl_gemv_stream.cu), M <= 16.
+struct StreamProblem {
+    const void* x;          // fused form: activations [M][K] (fp32/bf16)
+    const int8_t* q;        // unfused form: int8 [M][Kp]
+    const float* s;         // unfused form: fp32 [M]
+    const uint8_t* packed;
+    const float* gamma32;
+    void* y;
+    int32_t* acc;           // optional
+    int64_t N, K;
+    int cta_begin;          // set by plan_stream
+    int ctas;               // set by plan_stream
+};
+struct StreamBatch {
+    StreamProblem p[kMaxGroup];
+    int count;
+    int M;
+    int stages;             // set by plan_stream
+    int q_bytes;            // set by plan_stream
+};
+constexpr int kMaxStages = 12;
+// dynamic shared memory per CTA for `minb` resident CTAs per SM
+constexpr int stream_budget(int minb) { return minb >= 4 ? 54 * 1024 : 110 * 1024; }
+int stream_tokens(int64_t M);
+int sm_count();
+bool plan_stream(StreamBatch& b, int minb, int* grid, size_t* smem);
+// Returns cudaErrorNotSupported if the shapes do not fit (shared memory).
+cudaError_t launch_stream(StreamBatch& b, bool fused, bl_dtype xt, bl_dtype yt, unsigned* status,
+                          cudaStream_t st);
+
 // Prefill tensor-core GEMM (tcgen05 kind::i8).  Returns cudaErrorNotSupported
 // when the shape is outside what the kernel handles; the caller then uses
 // the decode kernel.
 cudaError_t launch_gemm_tc(const int8_t* q, const float* s, const uint8_t* packed,
                            const float* gamma32, int64_t M, int64_t N, int64_t K, void* y,
-                           bl_dtype yt, int32_t* acc, cudaStream_t st);
+                           bl_dtype yt, int32_t* acc, unsigned* status, cudaStream_t st);
 bool gemm_tc_supported(int64_t M, int64_t N, int64_t K);
 
 }  // namespace bl
