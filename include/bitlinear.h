@@ -99,6 +99,36 @@ bl_status bitlinear_pack_weights(const float* W, int64_t N, int64_t K, double ep
                                  void* workspace, size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
+ * bitlinear_pack_weights_noalloc -- bitlinear_pack_weights without the
+ * workspace argument.  The BitNet pages have no counterpart to this call;
+ * it is an interface addition of this library.
+ *
+ * For callers that cannot allocate device memory where they call the
+ * packer: for example a host framework's custom-operator hook that hands
+ * over its tensors but no allocator, or a deployment that reserves all
+ * device memory when it starts and forbids cudaMalloc afterwards (a
+ * cudaMalloc can synchronise the device and breaks a fixed memory plan).
+ *
+ * Arguments, results and errors are those of bitlinear_pack_weights minus
+ * the workspace.  The reduction's fp64 partial sums live instead in a
+ * fixed 16,640-byte array of the library's own device memory, which every
+ * GPU that loads the library holds until the process exits.
+ *   - Nothing is allocated: no cudaMalloc/cudaFree, no allocating library.
+ *   - The first call on a device looks up the array's device address (with
+ *     that device current) and caches it; make that first call before any
+ *     stream capture.
+ *   - Every call on a device uses the same array, so calls whose kernels
+ *     overlap on the GPU (different streams with no ordering between them)
+ *     race and give wrong results: order them on one stream or with events.
+ *   - A size whose scratch would not fit the array returns
+ *     BL_ERR_WORKSPACE; the reduction's block count is capped at 2048, so
+ *     every N, K accepted by bitlinear_pack_weights fits.
+ * ---------------------------------------------------------------------- */
+bl_status bitlinear_pack_weights_noalloc(const float* W, int64_t N, int64_t K, double eps,
+                                         uint8_t* packed, double* gamma64, float* gamma32,
+                                         void* stream);
+
+/* ------------------------------------------------------------------------
  * bitlinear_quant_act -- per-token absmax int8 quantisation (aratech.ae,
  * "BitLinear: the building block": each token's largest |activation| is
  * mapped to 127).

@@ -28,6 +28,7 @@ SIGNATURES = {
     "bitlinear_packed_bytes": (_i64, [_i64, _i64]),
     "bitlinear_pack_workspace_bytes": (_i64, [_i64, _i64]),
     "bitlinear_pack_weights": (_i32, [_vp, _i64, _i64, C.c_double, _vp, _vp, _vp, _vp, C.c_size_t, _vp]),
+    "bitlinear_pack_weights_noalloc": (_i32, [_vp, _i64, _i64, C.c_double, _vp, _vp, _vp, _vp]),
     "bitlinear_quant_act": (_i32, [_vp, _i32, _i64, _i64, _vp, _vp, _vp]),
     "bitlinear_forward": (_i32, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _i32, _vp, _vp]),
     "bitlinear_forward_x": (_i32, [_vp, _i32, _vp, _vp, _i64, _i64, _i64, _vp, _i32, _vp]),
@@ -123,6 +124,16 @@ def bitlinear_pack_weights(W, eps, packed, gamma64, gamma32, workspace, stream=N
                                       _dptr(workspace, "workspace"), workspace.numel() * workspace.element_size(),
                                       _stream(stream))
     _check(st, "bitlinear_pack_weights")
+
+
+def bitlinear_pack_weights_noalloc(W, eps, packed, gamma64, gamma32, stream=None) -> None:
+    """bitlinear_pack_weights with its scratch in the library's own fixed
+    device array: for callers that cannot allocate device memory."""
+    N, K = W.shape
+    st = lib().bitlinear_pack_weights_noalloc(_dptr(W, "W"), N, K, float(eps), _dptr(packed, "packed"),
+                                              _dptr(gamma64, "gamma64"), _dptr(gamma32, "gamma32"),
+                                              _stream(stream))
+    _check(st, "bitlinear_pack_weights_noalloc")
 
 
 def bitlinear_quant_act(x, q, s, stream=None) -> None:

@@ -41,6 +41,10 @@ bl_status check_forward_shape(int64_t M, int64_t N, int64_t K)
 
 }  // namespace
 
+namespace bl {
+unsigned* status_word_ptr() { return status_word(); }
+}  // namespace bl
+
 extern "C" {
 
 int64_t bitlinear_padded_k(int64_t K) { return K <= 0 ? 0 : bl::padded_k(K); }

@@ -27,6 +27,9 @@ __host__ __device__ inline int64_t tile_bytes(int64_t K) { return chunks_per_row
 constexpr unsigned kStatusNonfiniteW = 1u;
 constexpr unsigned kStatusNonfiniteX = 2u;
 
+// Device address of the current device's status word (NULL on failure).
+unsigned* status_word_ptr();
+
 // ---- launch helpers (host side, one per .cu file) ------------------------
 // Each returns cudaSuccess or the launch error; validation is done by the
 // caller in bl_api.cu.
