@@ -18,7 +18,9 @@ the data path), timed as the max over ranks.
 
 Other workloads (--workload): 7b (decode at 7B-class shapes, --m 1/4/16),
 prefill (M = 2048 tokens on the tensor cores; metric int8 TOPS), pack
-(absmean quantise + 2-bit pack of the block's weights).
+(absmean quantise + 2-bit pack of the block's weights), sweep100b (one token
+through 80 layers x 7 linears of a 100B-class model, 17.1 GB of packed
+weights resident; weights drawn on the GPU by the counter-based generator).
 
 --impl reference times the CPU oracle (oracle/, plain C) on the same
 workload and metric, on this machine's host cores.
@@ -48,7 +50,7 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=4000)
     ap.add_argument("--warmup", type=int, default=200)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["block2b", "7b", "prefill", "pack"], default="block2b")
+    ap.add_argument("--workload", choices=["block2b", "7b", "prefill", "pack", "sweep100b"], default="block2b")
     ap.add_argument("--m", type=int, default=1, help="tokens for --workload 7b")
     ap.add_argument("--mode", choices=["grouped", "fused", "separate"], default="grouped",
                     help="decode: grouped = one launch per step; fused = one launch per linear; "
@@ -500,6 +502,65 @@ def run_pack(torch, bl, args, dev, stream, dist, l2):
                     "for weights that fit there"}
 
 
+SWEEP_SEED = 1234
+
+
+def run_sweep(torch, bl, args, dev, stream, dist):
+    """80 layers x 7 linears at M = 1; one grouped fused launch per layer."""
+    import numpy as np
+    import synth
+    import synth.device as sd
+    kmax = max(K * N for K, N, _ in synth.LAYER100B)
+    wbuf = torch.empty(kmax, dtype=torch.float32, device=dev)
+    layers = []
+    t0 = time.perf_counter()
+    for layer in range(synth.LAYERS100B):
+        ps, gs, xs, ys = [], [], [], []
+        for j, (K, N, name) in enumerate(synth.LAYER100B):
+            g = layer * 7 + j
+            W = wbuf[:N * K].view(N, K)
+            sd.weights(W, SWEEP_SEED, g, 0, stream.cuda_stream)
+            p = torch.empty(bl.bitlinear_packed_bytes(N, K), dtype=torch.uint8, device=dev)
+            g64 = torch.empty(1, dtype=torch.float64, device=dev)
+            g32 = torch.empty(1, dtype=torch.float32, device=dev)
+            ws = torch.empty(bl.bitlinear_pack_workspace_bytes(N, K), dtype=torch.uint8, device=dev)
+            bl.bitlinear_pack_weights(W, 1e-5, p, g64, g32, ws, stream)
+            x = synth.activations(1, K, 50_000 + g, "bf16")
+            ps.append(p)
+            gs.append(g32)
+            xs.append(torch.from_numpy(x.view(np.int16)).to(dev).view(torch.bfloat16))
+            ys.append(torch.empty((1, N), dtype=torch.float32, device=dev))
+        layers.append((xs, ps, gs, ys))
+    torch.cuda.synchronize()
+    setup_s = time.perf_counter() - t0
+    del wbuf
+    if bl.bitlinear_get_status() != bl.BL_OK:
+        raise RuntimeError("non-finite weights")
+    Ns = [N for K, N, _ in synth.LAYER100B]
+    Ks = [K for K, N, _ in synth.LAYER100B]
+
+    def step(i):
+        for xs, ps, gs, ys in layers:
+            bl.bitlinear_forward_x_grouped(xs, ps, gs, Ns, Ks, ys, stream)
+
+    step(0)
+    torch.cuda.synchronize()
+    G = Graphs(torch, stream, step, 1)
+    G.run(max(3, min(args.warmup, 10)))
+    steps = max(3, min(args.steps, 50))
+    sampler = ClockSampler(dev.index)
+    sampler.start()
+    ms = time_region(torch, stream, lambda: G.run(steps), dist, dev)
+    clocks = sampler.stop()
+    if bl.bitlinear_get_status() != bl.BL_OK:
+        raise RuntimeError("device status word set during the timed region")
+    lin = [dict(K=K, N=N) for K, N, _ in synth.LAYER100B]
+    nbytes = decode_bytes(lin, 1) * synth.LAYERS100B
+    packed_bytes = sum(p.numel() for _, ps, _, _ in layers for p in ps)
+    return dict(ms=ms, steps=steps, nbytes=nbytes, packed_bytes=packed_bytes, clocks=clocks, setup_s=setup_s,
+                launches=synth.LAYERS100B)
+
+
 def main():
     args = parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -547,6 +608,23 @@ def main():
                "clocks": clocks}
         if rank == 0 and not args.no_cpu_baseline:
             out["cpu_baseline"] = cpu_baseline(lin, args.cpu_seconds, prefill=True)
+    elif args.workload == "sweep100b":
+        R = run_sweep(torch, bl, args, dev, stream, dist)
+        per_step = R["ms"] / R["steps"]
+        value = R["nbytes"] * R["steps"] * world / (R["ms"] / 1e3) / 1e9
+        achieved = R["nbytes"] / (per_step / 1e3) / 1e9
+        out = {"metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": R["steps"],
+               "warmup": args.warmup, "ms_per_step": per_step, "higher_is_better": True, "scaling": "weak",
+               "vs_baseline": None, "dtype": "int32", "data": "synthetic",
+               "config": {"workload": "sweep100b_decode_m1", "layers": 80,
+                          "linears": [f"{K}->{N}" for K, N, _ in __import__("synth").LAYER100B],
+                          "resident_packed_bytes": R["packed_bytes"], "setup_s": R["setup_s"],
+                          "l2_policy": "inputs larger than L2 (17.1 GB resident, streamed once per step)"},
+               "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                            "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                            "kernel": "stream_kernel (80 grouped launches per step)",
+                            "avg_launch_us": per_step / R["launches"] * 1e3},
+               "gpu_launches": R["launches"] * R["steps"], "clocks": R["clocks"]}
     elif args.workload == "pack":
         pk = run_pack(torch, bl, args, dev, stream, dist, l2)
         out = {"metric": "absmean ternary quantise + 2-bit pack, GB/s", "value": pk["value"] * world,

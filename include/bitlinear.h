@@ -52,7 +52,8 @@ typedef enum {
     BL_ERR_OVERFLOW = 6,    /* 127 * K >= 2^31: int32 accumulator could overflow   */
     BL_ERR_NONFINITE = 7,   /* device saw NaN/Inf in W or x (from get_status)      */
     BL_ERR_CUDA = 8,        /* a CUDA runtime call or kernel launch failed          */
-    BL_ERR_ARG = 9          /* another argument is invalid (eps < 0, count <= 0)   */
+    BL_ERR_ARG = 9,         /* another argument is invalid (eps < 0, count <= 0)   */
+    BL_ERR_TIMEOUT = 10     /* a kernel gave up a bounded wait (from get_status)    */
 } bl_status;
 
 typedef enum { BL_F32 = 0, BL_BF16 = 1 } bl_dtype;
@@ -189,8 +190,9 @@ bl_status bitlinear_forward_x_grouped(int count, const void* const* x, bl_dtype 
                                       void* const* y, bl_dtype yt, void* stream);
 
 /* Synchronises `stream`, then returns and clears the device status word of
- * the current device: BL_OK, or BL_ERR_NONFINITE if a kernel met NaN/Inf.
- * Returns BL_ERR_CUDA if the synchronisation itself failed. */
+ * the current device: BL_OK; BL_ERR_TIMEOUT if a kernel abandoned one of its
+ * bounded waits (its outputs are then invalid); else BL_ERR_NONFINITE if a
+ * kernel met NaN/Inf.  Returns BL_ERR_CUDA if the synchronisation failed. */
 bl_status bitlinear_get_status(void* stream);
 
 /* Static, human-readable name of a status value (never NULL). */

@@ -18,7 +18,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libbitlinear.so")
 
 BL_OK, BL_ERR_NULL, BL_ERR_SHAPE, BL_ERR_ALIGN, BL_ERR_DTYPE = 0, 1, 2, 3, 4
-BL_ERR_WORKSPACE, BL_ERR_OVERFLOW, BL_ERR_NONFINITE, BL_ERR_CUDA, BL_ERR_ARG = 5, 6, 7, 8, 9
+BL_ERR_WORKSPACE, BL_ERR_OVERFLOW, BL_ERR_NONFINITE, BL_ERR_CUDA, BL_ERR_ARG, BL_ERR_TIMEOUT = 5, 6, 7, 8, 9, 10
 BL_F32, BL_BF16 = 0, 1
 
 # Every symbol include/bitlinear.h declares, with (restype, argtypes).

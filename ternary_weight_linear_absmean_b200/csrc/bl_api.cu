@@ -4,6 +4,7 @@
 #include <cstring>
 
 #include "bl_internal.cuh"
+#include "bl_ptx.cuh"
 
 // One status word per device (the only global state of the library).
 __device__ unsigned int g_bl_status_word;
@@ -214,7 +215,7 @@ bl_status bitlinear_get_status(void* stream)
     if (v != 0) {
         const unsigned zero = 0;
         if (cudaMemcpyToSymbol(g_bl_status_word, &zero, sizeof(zero)) != cudaSuccess) return BL_ERR_CUDA;
-        return BL_ERR_NONFINITE;
+        return (v & bl::kStatusTimeout) ? BL_ERR_TIMEOUT : BL_ERR_NONFINITE;
     }
     return BL_OK;
 }
@@ -232,6 +233,7 @@ const char* bitlinear_status_string(bl_status status)
         case BL_ERR_NONFINITE: return "BL_ERR_NONFINITE: NaN or Inf met in W or x";
         case BL_ERR_CUDA: return "BL_ERR_CUDA: a CUDA call or kernel launch failed";
         case BL_ERR_ARG: return "BL_ERR_ARG: invalid argument";
+        case BL_ERR_TIMEOUT: return "BL_ERR_TIMEOUT: a kernel abandoned a bounded wait; outputs are invalid";
     }
     return "unknown bl_status";
 }

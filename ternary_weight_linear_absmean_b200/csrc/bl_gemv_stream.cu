@@ -17,8 +17,8 @@
 //                   form) or copy q there, while the first stages are in
 //                   flight; then for each stage take 512-byte spans (4 chunks
 //                   x 8 rows of a tile) round-robin, lane l reading 16 bytes,
-//                   row r = l % 8, and accumulate with dp4a (decode as in
-//                   bl_gemv.cu).  Per-lane partial sums are added into a
+//                   row r = l % 8, and accumulate with signed dp4a (decode
+//                   as in bl_gemv.cu).  Per-lane partial sums are added into a
 //                   per-(tile, row, token) int32 array in shared memory
 //                   (integer adds: exact and order-independent) whenever the
 //                   lane's tile changes.
@@ -73,70 +73,104 @@ __device__ __forceinline__ int consumers_sum(int v, int* red)
     return t;
 }
 
+__device__ __forceinline__ int consumers_max_int(int v, int* red)
+{
+    for (int o = 16; o > 0; o >>= 1) v = max(v, __shfl_xor_sync(0xffffffffu, v, o));
+    const int cw = (threadIdx.x >> 5) - 1;
+    if ((threadIdx.x & 31) == 0) red[cw] = v;
+    named_bar(1, kConsumers);
+    int m = red[0];
+#pragma unroll
+    for (int w = 1; w < kConsumerWarps; ++w) m = max(m, red[w]);
+    named_bar(1, kConsumers);   // red is reused right after
+    return m;
+}
+
+// four int32 codes in [-127, 127] -> one packed int8x4 word
+__device__ __forceinline__ uint32_t pack4(int a, int b, int c, int d)
+{
+    return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
+}
+
 // Quantise x row (K elements) into q (Kp bytes) in shared memory; returns s.
 // Same arithmetic as bl_quant.cu: amax over the row, s = 127 / max(amax,
-// 1e-5) (IEEE divide), q = clamp(rint(x * s), -127, 127) in fp32.
+// 1e-5) (IEEE divide), q = clamp(rint(x * s), -127, 127) in fp32.  Two
+// exact shortcuts: (1) max|x| is taken as an unsigned max over the bit
+// patterns with the sign cleared -- for non-negative IEEE values integer
+// order is numeric order, and NaN/Inf patterns sort above every finite
+// value, so the same max also flags non-finite input; (2) rint + clamp +
+// convert is one round-to-nearest-even conversion, since |x * s| < 127.5
+// for finite x (the clamp can never bind).
 template <typename XT>
-__device__ float quantise_row(const XT* __restrict__ row, int K, int Kp, int8_t* q, float* redf, int* redi,
-                              int* sumq_out, unsigned* status)
+__device__ float quantise_row(const XT* __restrict__ row, int K, int Kp, int8_t* q, int* redi, int* sumq_out,
+                              unsigned* status)
 {
     const int t = threadIdx.x - 32;
+    constexpr bool BF16 = sizeof(XT) == 2;
     constexpr int VE = 16 / sizeof(XT);   // elements per 16-byte vector
     const bool vec = (K % VE) == 0;
-    float amax = 0.0f;
-    bool bad = false;
+    uint32_t mbits = 0;                   // max |x| bit pattern (fp32 layout)
     if (vec) {
         const uint4* rv = reinterpret_cast<const uint4*>(row);
+        uint32_t mhi = 0, mlo = 0;
         for (int v = t; v < K / VE; v += kConsumers) {
             const uint4 u = __ldg(rv + v);
-            const XT* e = reinterpret_cast<const XT*>(&u);
+            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-            for (int i = 0; i < VE; ++i) {
-                const float f = to_f(e[i]);
-                bad |= !isfinite(f);
-                amax = fmaxf(amax, fabsf(f));
+            for (int i = 0; i < 4; ++i) {
+                if constexpr (BF16) {
+                    mhi = max(mhi, w[i] & 0x7FFF0000u);
+                    mlo = max(mlo, (w[i] << 16) & 0x7FFF0000u);
+                } else {
+                    mhi = max(mhi, w[i] & 0x7FFFFFFFu);
+                }
             }
         }
+        mbits = max(mhi, mlo);
     } else {
-        for (int k = t; k < K; k += kConsumers) {
-            const float f = to_f(row[k]);
-            bad |= !isfinite(f);
-            amax = fmaxf(amax, fabsf(f));
-        }
+        for (int k = t; k < K; k += kConsumers) mbits = max(mbits, __float_as_uint(to_f(row[k])) & 0x7FFFFFFFu);
     }
-    if (bad) atomicOr(status, kStatusNonfiniteX);
-    amax = fmaxf(consumers_max(amax, redf), 1e-5f);
+    mbits = (uint32_t)consumers_max_int((int)mbits, redi);
+    if (mbits >= 0x7F800000u && t == 0) atomicOr(status, kStatusNonfiniteX);
+    const float amax = fmaxf(__uint_as_float(mbits), 1e-5f);
     const float s = 127.0f / amax;
     int part = 0;
     if (vec) {
         const uint4* rv = reinterpret_cast<const uint4*>(row);
         for (int v = t; v < K / VE; v += kConsumers) {
             const uint4 u = __ldg(rv + v);
-            const XT* e = reinterpret_cast<const XT*>(&u);
-            uint32_t words[VE / 4];
+            if constexpr (BF16) {
+                const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+                int c[8];
 #pragma unroll
-            for (int w = 0; w < VE / 4; ++w) {
-                uint32_t word = 0;
-#pragma unroll
-                for (int b = 0; b < 4; ++b) word |= (uint32_t)(uint8_t)quant_one(to_f(e[4 * w + b]), s) << (8 * b);
-                words[w] = word;
-                part = dp4a_ss(word, 0x01010101u, part);
+                for (int i = 0; i < 4; ++i) {
+                    c[2 * i] = __float2int_rn(__fmul_rn(__uint_as_float(w[i] << 16), s));
+                    c[2 * i + 1] = __float2int_rn(__fmul_rn(__uint_as_float(w[i] & 0xFFFF0000u), s));
+                }
+                const uint32_t p0 = pack4(c[0], c[1], c[2], c[3]);
+                const uint32_t p1 = pack4(c[4], c[5], c[6], c[7]);
+                part = dp4a_ss(p0, 0x01010101u, part);
+                part = dp4a_ss(p1, 0x01010101u, part);
+                *reinterpret_cast<uint2*>(q + v * 8) = make_uint2(p0, p1);
+            } else {
+                const uint32_t p0 = pack4(__float2int_rn(__fmul_rn(__uint_as_float(u.x), s)),
+                                          __float2int_rn(__fmul_rn(__uint_as_float(u.y), s)),
+                                          __float2int_rn(__fmul_rn(__uint_as_float(u.z), s)),
+                                          __float2int_rn(__fmul_rn(__uint_as_float(u.w), s)));
+                part = dp4a_ss(p0, 0x01010101u, part);
+                *reinterpret_cast<uint32_t*>(q + v * 4) = p0;
             }
-            if constexpr (VE == 8)
-                *reinterpret_cast<uint2*>(q + v * 8) = make_uint2(words[0], words[1]);
-            else
-                *reinterpret_cast<uint32_t*>(q + v * 4) = words[0];
         }
         for (int k4 = K + 4 * t; k4 < Kp; k4 += 4 * kConsumers) *reinterpret_cast<uint32_t*>(q + k4) = 0u;
     } else {
         for (int k4 = 4 * t; k4 < Kp; k4 += 4 * kConsumers) {
-            uint32_t word = 0;
+            int c[4];
 #pragma unroll
             for (int b = 0; b < 4; ++b) {
                 const int k = k4 + b;
-                const int8_t v = (k < K) ? quant_one(to_f(row[k]), s) : (int8_t)0;
-                word |= (uint32_t)(uint8_t)v << (8 * b);
+                c[b] = (k < K) ? __float2int_rn(__fmul_rn(to_f(row[k]), s)) : 0;
             }
+            const uint32_t word = pack4(c[0], c[1], c[2], c[3]);
             *reinterpret_cast<uint32_t*>(q + k4) = word;
             part = dp4a_ss(word, 0x01010101u, part);
         }
@@ -156,10 +190,10 @@ __device__ __forceinline__ void dot_chunk(const uint4 wv, const int8_t* qs, int 
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const uint4 a = a4[i];
-                acc[m][0] = dp4a_us(U[i] & 0x03030303u, a.x, acc[m][0]);
-                acc[m][1] = dp4a_us(U[i] & 0x0C0C0C0Cu, a.y, acc[m][1]);
-                acc[m][2] = dp4a_us(U[i] & 0x30303030u, a.z, acc[m][2]);
-                acc[m][3] = dp4a_us(U[i] & 0xC0C0C0C0u, a.w, acc[m][3]);
+                acc[m][0] = dp4a_ss(U[i] & 0x03030303u, a.x, acc[m][0]);
+                acc[m][1] = dp4a_ss(U[i] & 0x0C0C0C0Cu, a.y, acc[m][1]);
+                acc[m][2] = dp4a_ss(U[i] & 0x30303030u, a.z, acc[m][2]);
+                acc[m][3] = dp4a_ss((U[i] >> 2) & 0x30303030u, a.w, acc[m][3]);
             }
         }
     }
@@ -176,6 +210,7 @@ stream_kernel(const __grid_constant__ StreamBatch b, unsigned* status)
     __shared__ float redf[kConsumerWarps];
     __shared__ int redi[kConsumerWarps];
     __shared__ int abort_flag;
+    __shared__ int piece_ok[2];
 
     // ---- which problem, which tiles
     int pi = 0;
@@ -240,7 +275,7 @@ stream_kernel(const __grid_constant__ StreamBatch b, unsigned* status)
 #pragma unroll 1
         for (int m = 0; m < M; ++m) {
             int sq;
-            const float s = quantise_row<XT>(xb + (int64_t)m * K, K, Kp, qs + m * Kp, redf, redi, &sq, status);
+            const float s = quantise_row<XT>(xb + (int64_t)m * K, K, Kp, qs + m * Kp, redi, &sq, status);
             if (threadIdx.x == 32) {
                 s_scale[m] = s;
                 s_sumq[m] = sq;
@@ -283,7 +318,7 @@ stream_kernel(const __grid_constant__ StreamBatch b, unsigned* status)
 #pragma unroll
             for (int m = 0; m < MT; ++m) {
                 if (m < M) {
-                    const int tot = acc[m][0] + (acc[m][1] >> 2) + (acc[m][2] >> 4) + (acc[m][3] >> 6);
+                    const int tot = acc[m][0] + (acc[m][1] >> 2) + (acc[m][2] >> 4) + (acc[m][3] >> 4);
                     atomicAdd(&sacc[(cur * 8 + r) * MT + m], tot);
                 }
 #pragma unroll
@@ -296,7 +331,19 @@ stream_kernel(const __grid_constant__ StreamBatch b, unsigned* status)
 #pragma unroll 1
     for (int j = 0; j < npieces; ++j) {
         const int s = j % stages, round = j / stages;
-        if (!wait_parity(&full_bar[s], round & 1, status, &abort_flag)) break;
+        // one consumer warp polls the stage barrier; the others sleep in a
+        // hardware named barrier, then confirm the (already complete) phase
+        // themselves, which gives every thread its own acquire of the data.
+        // The outcome is published in piece_ok[j & 1] before the barrier so
+        // that every consumer warp takes the same branch (a warp missing a
+        // later named barrier would leave the others waiting forever).
+        if (cw == 0) {
+            const bool ok = wait_parity(&full_bar[s], round & 1, status, &abort_flag);
+            if (lane == 0) piece_ok[j & 1] = ok && !abort_flag;
+        }
+        named_bar(2, kConsumers);
+        if (!piece_ok[j & 1]) break;
+        mbar_try_wait(&full_bar[s], round & 1);   // completed phase: this thread's acquire
         const uint32_t poff = (uint32_t)j * kStageBytes;
         const uint32_t len = (range - poff) < (uint32_t)kStageBytes ? (range - poff) : (uint32_t)kStageBytes;
         const uint8_t* stage = ring + (size_t)s * kStageBytes;

@@ -58,15 +58,35 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity)
     return ok != 0;
 }
 
-// Bounded wait for the phase with the given parity to complete.  Returns
-// false (and flags the status word) on timeout or if *abort is raised.
+// try_wait with a suspend-time hint: the thread may sleep (not issue) until
+// the phase completes or about `ns` nanoseconds pass.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t ns)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(ns)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait for the phase with the given parity to complete, polling
+// with exponential __nanosleep back-off (32 .. 512 ns) so waiting warps take
+// few issue slots.  Returns false (and flags the status word) on timeout or
+// if *abort is raised.
 __device__ __forceinline__ bool wait_parity(uint64_t* bar, uint32_t parity, unsigned* status,
                                            volatile int* abort)
 {
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
+    unsigned ns = 32;
     while (true) {
-        if (mbar_try_wait(bar, parity)) return true;
+        if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
+        __nanosleep(ns);                       // back off: a polling warp issues nothing while asleep
+        if (ns < 512) ns <<= 1;
         if (abort && *abort) return false;
         if (clock64() - t0 > kWaitCycles) {
             if (status) atomicOr(status, kStatusTimeout);

@@ -48,7 +48,7 @@ def test_size_functions_match_layout_spec(L):
 
 
 def test_status_strings(L):
-    for s in range(10):
+    for s in range(11):
         assert bl.status_string(s).startswith("BL_")
     assert "unknown" in bl.status_string(99)
 
