@@ -136,10 +136,13 @@ def decode_bytes(lin, M):
 
 
 def max_over_ranks(ms, dist, dev):
+    """The slowest rank's time: every rank contributes its own CUDA-event
+    time and all take the maximum (dev=None reduces on the CPU, as with a
+    gloo group)."""
     if dist is None:
         return ms
     import torch
-    t = torch.tensor([ms], device=dev, dtype=torch.float64)
+    t = torch.tensor([ms], device=dev if dev is not None else "cpu", dtype=torch.float64)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 

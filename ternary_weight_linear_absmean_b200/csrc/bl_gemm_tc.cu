@@ -5,21 +5,29 @@
 // integer adds; aratech.ae "BitLinear: the building block" for the int8
 // per-token activations.)
 //
-// Tile: 128 weight rows (MMA M) x 256 tokens (MMA N) per CTA, K in stages of
-// 128.  The weights never exist as int8 in memory: the packed 2-bit codes
-// are TMA-loaded (4 KiB per stage), four expansion warps decode them to
-// signed int8 in registers and write them straight into tensor memory with
+// Persistent kernel, one CTA per SM, looping over 128 (weight rows, MMA M)
+// x 128 (tokens, MMA N) output tiles; K in stages of 128, 8 stages deep.
+// The weights never exist as int8 in memory: the packed 2-bit codes are
+// TMA-loaded (4 KiB per stage), eight expansion warps decode them to signed
+// int8 in registers and write them straight into tensor memory with
 // tcgen05.st, where the MMA reads them as its A operand.  Shared memory only
 // carries the activation tiles (B operand, TMA with 128-byte swizzle).
 //
-// Warp roles (256 threads):
-//   warp 0      TMEM allocation; TMA producer (one lane)
-//   warp 1      MMA issuer (one lane): 4 x tcgen05.mma (K = 32) per stage,
-//               tcgen05.commit -> stage-free barrier, final commit -> accum
-//   warps 2-3   per-token rescale factors gamma32 / s_m (fp64)
-//   warps 4-7   expansion (TMEM lanes 32*(w-4) ..), then the epilogue:
-//               tcgen05.ld of the accumulator, rescale, store y
-// All mbarrier waits are bounded (bl_ptx.cuh).
+// Tensor memory (512 columns): two 128-column int32 accumulators (tile i is
+// drained by the epilogue while tile i+1 accumulates into the other) and
+// eight 32-column A stages.
+//
+// Warp roles (512 threads):
+//   warp 0       TMEM allocation; TMA producer (one lane)
+//   warp 1       MMA issuer (one lane): 4 x tcgen05.mma (K = 32) per stage,
+//                tcgen05.commit -> stage-free barrier; per tile -> acc-full
+//   warps 4-11   expansion, two groups of four taking alternate stages:
+//                warp w writes TMEM lanes 32*(w%4) .. +31 of its stages
+//   warps 12-15  epilogue: per-token factors gamma32 / s_m (fp64),
+//                tcgen05.ld of the finished accumulator, rescale, store y,
+//                then release the accumulator
+// All mbarrier waits are bounded (bl_ptx.cuh); every role reaches the final
+// barrier, after which the allocating warp frees the tensor memory.
 //
 // Decode to signed int8: per 2-bit field (lo, hi), code = lo - hi.
 //   S = (w & 0x55555555 | 0xAAAAAAAA) - ((w >> 1) & 0x55555555)
@@ -36,23 +44,27 @@ namespace bl {
 namespace {
 
 constexpr int BM = 128;        // weight rows per tile (MMA M)
-constexpr int BN = 256;        // tokens per tile (MMA N)
+constexpr int BN = 128;        // tokens per tile (MMA N)
 constexpr int BK = 128;        // k per stage (bytes of int8)
-constexpr int STAGES = 4;
-constexpr int kThreads = 256;
-constexpr int Q_STAGE = BN * BK;             // 32 KiB, 128B-swizzled
+constexpr int STAGES = 8;
+constexpr int kThreads = 512;
+constexpr int Q_STAGE = BN * BK;             // 16 KiB, 128B-swizzled
 constexpr int W_STAGE = (BM / 8) * 256;      // 16 tiles x 2 chunks x 128 B = 4 KiB
 constexpr int TMEM_COLS = 512;
-constexpr int A_COL0 = 256;                  // A stages after the accumulator
+constexpr int ACC_COLS = BN;                 // one accumulator buffer
+constexpr int A_COL0 = 2 * ACC_COLS;         // A stages after the two accumulators
 constexpr int A_STAGE_COLS = BK / 4;         // 32 columns per stage
+constexpr int EXP_WARP0 = 4, EPI_WARP0 = 12;
 
 struct Smem {
     uint8_t q[STAGES][Q_STAGE];              // 1024-aligned (first member)
     uint8_t w[STAGES][W_STAGE];
-    double fac[BN];
-    uint64_t full[STAGES], expanded[STAGES], empty[STAGES], accum;
+    double fac[2][BN];
+    uint64_t full[STAGES], expanded[STAGES], empty[STAGES];
+    uint64_t acc_full[2], acc_empty[2], done;
     uint32_t tmem_base;
     int abort_flag;
+    int epi_ok[2];
 };
 
 __device__ __forceinline__ uint32_t signed_codes(int t, uint32_t S)
@@ -72,7 +84,7 @@ __device__ __forceinline__ uint64_t make_bdesc(uint32_t smem_addr)
     return d;
 }
 
-// kind::i8, D = S32, A = B = signed int8, both K-major, M = 128, N = 256.
+// kind::i8, D = S32, A = B = signed int8, both K-major, M = 128, N = BN.
 constexpr uint32_t kIdesc = (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
                             ((uint32_t)(BM >> 4) << 24);
 
@@ -138,15 +150,20 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
     extern __shared__ uint8_t smem_raw[];
     Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int n0 = blockIdx.x * BM, m0 = blockIdx.y * BN;
+    const int tiles_n = (N + BM - 1) / BM, tiles_m = (M + BN - 1) / BN;
+    const int total = tiles_n * tiles_m;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&sm.full[s], 1);
-            mbar_init(&sm.expanded[s], 128);
+            mbar_init(&sm.expanded[s], 128);   // one expansion group
             mbar_init(&sm.empty[s], 1);
         }
-        mbar_init(&sm.accum, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&sm.acc_full[b], 1);
+            mbar_init(&sm.acc_empty[b], 128);
+        }
+        mbar_init(&sm.done, 1);
         sm.abort_flag = 0;
         fence_barrier_init();
     }
@@ -169,82 +186,122 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
         if (lane == 0) {
             prefetch_tmap(&tmap_q);
             prefetch_tmap(&tmap_w);
-            int issued = 0;
-            for (int kb = 0; kb < nk; ++kb) {
-                const int s = kb % STAGES, round = kb / STAGES;
-                if (round > 0 && !wait_parity(&sm.empty[s], (round - 1) & 1, status, abort)) break;
-                mbar_arrive_expect_tx(&sm.full[s], Q_STAGE + W_STAGE);
-                tma_load_2d(sm.q[s], &tmap_q, kb * BK, m0, &sm.full[s]);
-                tma_load_2d(sm.w[s], &tmap_w, kb * 256, n0 / 8, &sm.full[s]);
-                issued = kb + 1;
+            int g = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; ok && t < total; t += gridDim.x) {
+                const int n0 = (t % tiles_n) * BM, m0 = (t / tiles_n) * BN;
+                for (int kb = 0; kb < nk; ++kb, ++g) {
+                    const int s = g % STAGES, round = g / STAGES;
+                    if (round > 0 && !wait_parity(&sm.empty[s], (round - 1) & 1, status, abort)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&sm.full[s], Q_STAGE + W_STAGE);
+                    tma_load_2d(sm.q[s], &tmap_q, kb * BK, m0, &sm.full[s]);
+                    tma_load_2d(sm.w[s], &tmap_w, kb * 256, n0 / 8, &sm.full[s]);
+                }
             }
-            for (int kb = issued - STAGES < 0 ? 0 : issued - STAGES; kb < issued; ++kb)
-                wait_parity(&sm.full[kb % STAGES], (kb / STAGES) & 1, status, nullptr);
+            // every copy issued has landed before this thread leaves
+            for (int j = g - STAGES < 0 ? 0 : g - STAGES; j < g; ++j)
+                wait_parity(&sm.full[j % STAGES], (j / STAGES) & 1, status, nullptr, true);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            for (int kb = 0; kb < nk; ++kb) {
-                const int s = kb % STAGES;
-                const uint32_t ph = (kb / STAGES) & 1;
-                if (!wait_parity(&sm.full[s], ph, status, abort)) break;
-                if (!wait_parity(&sm.expanded[s], ph, status, abort)) break;
+            int g = 0, i = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; ok && t < total; t += gridDim.x, ++i) {
+                const int b = i & 1, ar = i >> 1;
+                if (ar > 0 && !wait_parity(&sm.acc_empty[b], (ar - 1) & 1, status, abort)) break;
                 tc_fence_after();
-                const uint32_t qaddr = smem_u32(sm.q[s]);
+                const uint32_t d_tmem = tmem + b * ACC_COLS;
+                for (int kb = 0; kb < nk; ++kb, ++g) {
+                    const int s = g % STAGES;
+                    const uint32_t ph = (g / STAGES) & 1;
+                    if (!wait_parity(&sm.full[s], ph, status, abort) ||
+                        !wait_parity(&sm.expanded[s], ph, status, abort)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t qaddr = smem_u32(sm.q[s]);
 #pragma unroll
-                for (int j = 0; j < BK / 32; ++j)
-                    mma_i8_ts(tmem, tmem + A_COL0 + s * A_STAGE_COLS + j * 8, make_bdesc(qaddr + j * 32),
-                              (kb | j) != 0);
-                mma_commit(&sm.empty[s]);
+                    for (int j = 0; j < BK / 32; ++j)
+                        mma_i8_ts(d_tmem, tmem + A_COL0 + s * A_STAGE_COLS + j * 8, make_bdesc(qaddr + j * 32),
+                                  (kb | j) != 0);
+                    mma_commit(&sm.empty[s]);
+                }
+                if (ok) mma_commit(&sm.acc_full[b]);
             }
-            mma_commit(&sm.accum);   // also on abort: retires every MMA issued
+            mma_commit(&sm.done);   // retires every MMA this thread issued
         }
-    } else if (warp < 4) {
-        // -------------------------------------------------- rescale factors
-        const double g = (double)*gamma32;
-        for (int j = threadIdx.x - 64; j < BN; j += 64) {
-            const int m = m0 + j;
-            sm.fac[j] = (m < M) ? g / (double)s_in[m] : 0.0;
-        }
-    } else {
-        // --------------------------------------------- expansion warps 4..7
-        const int rr = threadIdx.x - 128;          // TMEM lane = weight row in tile
-        const int quarter = warp - 4;
+    } else if (warp >= EXP_WARP0 && warp < EPI_WARP0) {
+        // --------------------------------------------- expansion warps 4..11
+        // Two groups of four warps take alternate stages, so each thread has
+        // two MMA-stage periods to decode, store into TMEM and wait for the
+        // store; the four warps of a group cover the 128 TMEM lanes.
+        const int quarter = warp & 3;
+        const int grp = (warp - EXP_WARP0) >> 2;               // stages g with g % 2 == grp
+        const int rr = 32 * quarter + lane;                    // TMEM lane = weight row in tile
         const uint32_t lane_base = (uint32_t)(32 * quarter) << 16;
         const int woff = (rr >> 3) * 256 + (rr & 7) * 16;
-        for (int kb = 0; kb < nk; ++kb) {
-            const int s = kb % STAGES;
-            const bool got = wait_parity(&sm.full[s], (kb / STAGES) & 1, status, abort);
-            if (!__all_sync(0xffffffffu, got)) break;   // warp-uniform: tcgen05.st is .aligned
-            uint32_t out[32];
-#pragma unroll
-            for (int cl = 0; cl < 2; ++cl) {
-                const uint4 wv = *reinterpret_cast<const uint4*>(sm.w[s] + woff + cl * 128);
-                const uint32_t words[4] = {wv.x, wv.y, wv.z, wv.w};
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const uint32_t w = words[i];
-                    const uint32_t S = ((w & 0x55555555u) | 0xAAAAAAAAu) - ((w >> 1) & 0x55555555u);
-#pragma unroll
-                    for (int t = 0; t < 4; ++t) out[16 * cl + 4 * i + t] = signed_codes(t, S);
+        int g = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; ok && t < total; t += gridDim.x) {
+            for (int kb = 0; kb < nk; ++kb, ++g) {
+                if ((g & 1) != grp) continue;
+                const int s = g % STAGES;
+                const bool got = wait_parity(&sm.full[s], (g / STAGES) & 1, status, abort);
+                if (!__all_sync(0xffffffffu, got)) {   // warp-uniform: tcgen05.st is .aligned
+                    ok = false;
+                    break;
                 }
+                uint32_t out[32];
+#pragma unroll
+                for (int cl = 0; cl < 2; ++cl) {
+                    const uint4 wv = *reinterpret_cast<const uint4*>(sm.w[s] + woff + cl * 128);
+                    const uint32_t words[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const uint32_t w = words[i];
+                        const uint32_t S = ((w & 0x55555555u) | 0xAAAAAAAAu) - ((w >> 1) & 0x55555555u);
+#pragma unroll
+                        for (int tt = 0; tt < 4; ++tt) out[16 * cl + 4 * i + tt] = signed_codes(tt, S);
+                    }
+                }
+                tmem_st32(tmem + lane_base + A_COL0 + s * A_STAGE_COLS, out);
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(&sm.expanded[s]);
             }
-            tmem_st32(tmem + lane_base + A_COL0 + s * A_STAGE_COLS, out);
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(&sm.expanded[s]);
         }
-        // ------------------------------------------------------- epilogue
-        __syncwarp();
-        named_bar(2, 128 + 64);   // factors ready (warps 2-7)
-        const bool ok = __all_sync(0xffffffffu, wait_parity(&sm.accum, 0, status, abort));
-        tc_fence_after();
-        const int n = n0 + rr;
-        if (ok) {
+    } else if (warp >= EPI_WARP0) {
+        // ------------------------------------------------ epilogue 12..15
+        const int et = threadIdx.x - 32 * EPI_WARP0;          // 0..127
+        const int quarter = warp & 3;
+        const int rr = 32 * quarter + lane;
+        const uint32_t lane_base = (uint32_t)(32 * quarter) << 16;
+        const double gam = (double)*gamma32;
+        int i = 0;
+        for (int t = blockIdx.x; t < total; t += gridDim.x, ++i) {
+            const int b = i & 1, ar = i >> 1;
+            const int n0 = (t % tiles_n) * BM, m0 = (t / tiles_n) * BN;
+            {
+                const int m = m0 + et;
+                sm.fac[b][et] = (m < M) ? gam / (double)s_in[m] : 0.0;
+            }
+            // one thread waits for the accumulator; the verdict goes through
+            // shared memory so all four warps take the same branch
+            if (et == 0) sm.epi_ok[b] = wait_parity(&sm.acc_full[b], ar & 1, status, abort, true) ? 1 : 0;
+            named_bar(3, 128);
+            if (!sm.epi_ok[b]) break;
+            tc_fence_after();
+            const int n = n0 + rr;
+            const uint32_t acc_tmem = tmem + lane_base + b * ACC_COLS;
 #pragma unroll 1
             for (int cc = 0; cc < BN / 32; ++cc) {
                 uint32_t v[32];
-                tmem_ld32(tmem + lane_base + cc * 32, v);
+                tmem_ld32(acc_tmem + cc * 32, v);
                 tmem_wait_ld();
                 if (n < N) {
 #pragma unroll
@@ -254,17 +311,18 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
                             const int a = (int)v[j];
                             const int64_t o = (int64_t)m * N + n;
                             if (acc_out) acc_out[o] = a;
-                            store_y(y, o, (float)((double)a * sm.fac[cc * 32 + j]));
+                            store_y(y, o, (float)((double)a * sm.fac[b][cc * 32 + j]));
                         }
                     }
                 }
             }
+            tc_fence_before();
+            mbar_arrive(&sm.acc_empty[b]);
         }
-        tc_fence_before();
     }
-    if (warp == 2 || warp == 3) named_bar(2, 128 + 64);
     __syncthreads();
     if (warp == 0) {
+        wait_parity(&sm.done, 0, status, nullptr, true);
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS)
                      : "memory");
@@ -313,7 +371,8 @@ cudaError_t launch_typed(const CUtensorMap& tq, const CUtensorMap& tw, const flo
         if (e != cudaSuccess) return e;
         configured[dev] = true;
     }
-    dim3 grid((N + BM - 1) / BM, (M + BN - 1) / BN);
+    const int tiles = ((N + BM - 1) / BM) * ((M + BN - 1) / BN);
+    const int grid = tiles < sm_count() ? tiles : sm_count();
     gemm_tc_kernel<YT><<<grid, kThreads, smem, st>>>(tq, tw, s, g, M, N, nk, static_cast<YT*>(y), acc, status);
     return cudaGetLastError();
 }
@@ -322,8 +381,9 @@ cudaError_t launch_typed(const CUtensorMap& tq, const CUtensorMap& tw, const flo
 
 bool gemm_tc_supported(int64_t M, int64_t N, int64_t K)
 {
-    return M > 16 && M < (int64_t(1) << 31) && N < (int64_t(1) << 31) && (M + BN - 1) / BN <= 65535 &&
-           padded_k(K) < (int64_t(1) << 31) && encode_fn() != nullptr;
+    return M > 16 && M < (int64_t(1) << 31) && N < (int64_t(1) << 31) &&
+           ((N + BM - 1) / BM) * ((M + BN - 1) / BN) < (int64_t(1) << 31) && padded_k(K) < (int64_t(1) << 31) &&
+           encode_fn() != nullptr;
 }
 
 cudaError_t launch_gemm_tc(const int8_t* q, const float* s, const uint8_t* packed, const float* gamma32,

@@ -179,13 +179,15 @@ __device__ float quantise_row(const XT* __restrict__ row, int K, int Kp, int8_t*
     return s;
 }
 
+// One 16-byte chunk (64 weights of row r) against the activations of chunk
+// c for every token slot; slots m >= M hold zero activations.
 template <int MT>
-__device__ __forceinline__ void dot_chunk(const uint4 wv, const int8_t* qs, int Kp, int c, int M, int (&acc)[MT][4])
+__device__ __forceinline__ void dot_chunk(const uint4 wv, const int8_t* qs, int Kp, int c, int (&acc)[MT][4])
 {
     const uint32_t U[4] = {biased_codes(wv.x), biased_codes(wv.y), biased_codes(wv.z), biased_codes(wv.w)};
 #pragma unroll
     for (int m = 0; m < MT; ++m) {
-        if (m < M) {
+        {
             const uint4* a4 = reinterpret_cast<const uint4*>(qs + m * Kp + c * 64);
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
@@ -305,7 +307,14 @@ stream_kernel(const __grid_constant__ StreamBatch b, unsigned* status)
         }
     }
 
+    // token slots M .. MT-1 get zero activations, so the dot loop needs no
+    // token guard (their sums are never written out)
+    for (int i = threadIdx.x - 32; i < (MT - M) * Kp / 16; i += kConsumers)
+        reinterpret_cast<uint4*>(qs + M * Kp)[i] = make_uint4(0, 0, 0, 0);
+    named_bar(1, kConsumers);
+
     const int r = lane & 7;
+    const int sub = lane >> 3;
     int cur = -1;
     int acc[MT][4];
 #pragma unroll
@@ -328,6 +337,8 @@ stream_kernel(const __grid_constant__ StreamBatch b, unsigned* status)
     };
 
     constexpr uint32_t kStep = kConsumerWarps * kSpan;   // bytes between a warp's spans
+    const bool aligned = (TB % kSpan) == 0;
+    const uint32_t spans_per_tile = TB / kSpan;
 #pragma unroll 1
     for (int j = 0; j < npieces; ++j) {
         const int s = j % stages, round = j / stages;
@@ -347,31 +358,56 @@ stream_kernel(const __grid_constant__ StreamBatch b, unsigned* status)
         const uint32_t poff = (uint32_t)j * kStageBytes;
         const uint32_t len = (range - poff) < (uint32_t)kStageBytes ? (range - poff) : (uint32_t)kStageBytes;
         const uint8_t* stage = ring + (size_t)s * kStageBytes;
-        // lane's position: one division per stage, then incremental
-        uint32_t boff = (uint32_t)cw * kSpan + (uint32_t)lane * 16;
-        uint32_t tile = (poff + boff) / TB;
-        uint32_t within = (poff + boff) - tile * TB;
-        uint4 wnext = make_uint4(0, 0, 0, 0);
-        if (boff < len) wnext = *reinterpret_cast<const uint4*>(stage + boff);
+        if (aligned) {
+            // Tiles are whole 512-byte spans: a span lies in one tile, so the
+            // tile index is the same for the whole warp and is tracked with
+            // one division per stage.
+            const uint32_t nsp = len / kSpan;
+            uint32_t gsp = poff / kSpan + (uint32_t)cw;        // span index in the CTA range
+            uint32_t tile = gsp / spans_per_tile;
+            uint32_t gin = gsp - tile * spans_per_tile;       // chunk group within the tile
+            const uint8_t* wp = stage + cw * kSpan + lane * 16;
 #pragma unroll 1
-        for (uint32_t sb = (uint32_t)cw * kSpan; sb < len; sb += kStep, boff += kStep) {
-            const uint4 wv = wnext;
-            if (boff + kStep < len) wnext = *reinterpret_cast<const uint4*>(stage + boff + kStep);
-            if (boff < len) {
+            for (uint32_t sp = (uint32_t)cw; sp < nsp; sp += kConsumerWarps, wp += kStep) {
                 if ((int)tile != cur) {
                     flush();
                     cur = (int)tile;
                 }
-                dot_chunk<MT>(wv, qs, Kp, (int)(within >> 7), M, acc);
-            }
-            within += kStep;
-            if (within >= TB) {
-                if (TB >= kStep) {
-                    within -= TB;
+                dot_chunk<MT>(*reinterpret_cast<const uint4*>(wp), qs, Kp, (int)(4 * gin) + sub, acc);
+                gin += kConsumerWarps;
+                if (gin >= spans_per_tile) {
+                    gin -= spans_per_tile;
                     ++tile;
-                } else {
-                    tile += within / TB;
-                    within %= TB;
+                    if (gin >= spans_per_tile) {
+                        tile += gin / spans_per_tile;
+                        gin %= spans_per_tile;
+                    }
+                }
+            }
+        } else {
+            // general case: a span may cross a tile boundary, so each lane
+            // tracks its own tile (one division per stage, then incremental)
+            uint32_t boff = (uint32_t)cw * kSpan + (uint32_t)lane * 16;
+            uint32_t tile = (poff + boff) / TB;
+            uint32_t within = (poff + boff) - tile * TB;
+#pragma unroll 1
+            for (uint32_t sb = (uint32_t)cw * kSpan; sb < len; sb += kStep, boff += kStep) {
+                if (boff < len) {
+                    if ((int)tile != cur) {
+                        flush();
+                        cur = (int)tile;
+                    }
+                    dot_chunk<MT>(*reinterpret_cast<const uint4*>(stage + boff), qs, Kp, (int)(within >> 7), acc);
+                }
+                within += kStep;
+                if (within >= TB) {
+                    if (TB >= kStep) {
+                        within -= TB;
+                        ++tile;
+                    } else {
+                        tile += within / TB;
+                        within %= TB;
+                    }
                 }
             }
         }

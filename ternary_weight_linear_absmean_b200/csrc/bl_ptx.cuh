@@ -73,20 +73,23 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t pari
     return ok != 0;
 }
 
-// Bounded wait for the phase with the given parity to complete, polling
-// with exponential __nanosleep back-off (32 .. 512 ns) so waiting warps take
-// few issue slots.  Returns false (and flags the status word) on timeout or
-// if *abort is raised.
+// Bounded wait for the phase with the given parity to complete.  Returns
+// false (and flags the status word) on timeout or if *abort is raised.
+// With `backoff` the poll sleeps (__nanosleep, 32 .. 256 ns) between tries,
+// so long waits by many warps take few issue slots; critical-path waiters
+// (MMA issuer, producers) poll without sleeping.
 __device__ __forceinline__ bool wait_parity(uint64_t* bar, uint32_t parity, unsigned* status,
-                                           volatile int* abort)
+                                           volatile int* abort, bool backoff = false)
 {
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
     unsigned ns = 32;
     while (true) {
         if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
-        __nanosleep(ns);                       // back off: a polling warp issues nothing while asleep
-        if (ns < 512) ns <<= 1;
+        if (backoff) {
+            __nanosleep(ns);
+            if (ns < 256) ns <<= 1;
+        }
         if (abort && *abort) return false;
         if (clock64() - t0 > kWaitCycles) {
             if (status) atomicOr(status, kStatusTimeout);
