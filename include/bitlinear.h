@@ -59,13 +59,14 @@ typedef enum {
 typedef enum { BL_F32 = 0, BL_BF16 = 1 } bl_dtype;
 
 /* ------------------------------------------------------------------------
- * Packed ternary weight layout (2 bits per weight, row-tiled, chunk-major).
- * Code values follow bhfrc.com/news/56965 sec. 4.1: 00 -> 0, 01 -> +1,
- * 10 -> -1, 11 -> padding (decodes to 0).
+ * Packed ternary weight layout (2 bits per weight, row-tiled, chunk-major;
+ * 2 bits per weight as in bhfrc.com/news/56965 sec. 4.1).  Each weight is
+ * stored as u = code + 1: 00 -> -1, 01 -> 0, 10 -> +1 (11 never occurs), so
+ * a decoder only masks fields out.  Padding holds 01 (code 0).
  *   Kp = ceil(K/64)*64, Np = ceil(N/8)*8, C = Kp/64 sixteen-byte chunks/row.
  *   Weight (n, k) sits in byte  (n/8)*(8*C*16) + ((k/64)*8 + n%8)*16
  *                                + ((k%64)/16)*4 + k%4
- *   at bits 2*((k%16)/4) .. +1.  Padded positions (n >= N or k >= K) hold 11.
+ *   at bits 2*((k%16)/4) .. +1.  Padded positions (n >= N or k >= K) hold 01.
  * So each 8-row tile stores chunk c of its 8 rows as 128 contiguous bytes,
  * and a warp reads 4 chunks x 8 rows as one 512-byte coalesced span.
  * ---------------------------------------------------------------------- */

@@ -13,8 +13,8 @@
  *             "Ternary weights {-1, 0, +1}" and "BitLinear: the building block".
  *   [BHFRC]   "BitNet b1.58 on Windows: sm_86 kernels + AVX2" build notes
  *             (bhfrc.com/news/56965, Chinese), sec. 1.1 (ternary weights turn
- *             each multiply into add / subtract / skip) and sec. 4.1 (2-bit
- *             code table 00 -> 0, 01 -> +1, 10 -> -1, 11 -> padding).
+ *             each multiply into add / subtract / skip) and sec. 4.1 (2 bits
+ *             per weight, packed for wide loads).
  *
  * Readings taken where the pages are silent (each also listed in the design doc):
  *   R1  eps = 1e-5 (caller-chosen), added to gamma in fp64, used only for the
@@ -81,9 +81,12 @@ int64_t orc_ternary_codes(const float* W, int64_t N, int64_t K, double gamma64,
 }
 
 /* ------------------------------------------------------------------------ */
-/* A2: 2-bit packed weight layout ("row-tiled, chunk-major").               */
-/* Code values follow [BHFRC] sec. 4.1: 00 -> 0, 01 -> +1, 10 -> -1,        */
-/* 11 -> padding (decodes to 0).                                            */
+/* A2: 2-bit packed weight layout ("row-tiled, chunk-major"), as specified */
+/* in include/bitlinear.h.  Each weight is stored as u = code + 1:           */
+/* 00 -> -1, 01 -> 0, 10 -> +1; padding is 01 (code 0); 11 never occurs.    */
+/* (The BitNet pages' CPU kernel ([BHFRC] sec. 4.1) uses a different 2-bit  */
+/* table, 00 -> 0, 01 -> +1, 10 -> -1, 11 -> padding; storing code + 1 is   */
+/* this layout's choice, so decoding needs masking only.)                   */
 /*                                                                          */
 /* Geometry (the library implements the same spec independently):          */
 /*   Kp = ceil(K / 64) * 64            padded reduction length              */
@@ -94,7 +97,7 @@ int64_t orc_ternary_codes(const float* W, int64_t N, int64_t K, double gamma64,
 /*   field t = (k % 16) / 4, byte b = k % 4                                 */
 /*   byte offset = tau * (8 * C * 16) + (c * 8 + r) * 16 + i * 4 + b        */
 /*   bit offset within that byte = 2 * t                                    */
-/* Padded positions (k >= K or n >= N) hold 11.                             */
+/* Padded positions (k >= K or n >= N) hold 01.                             */
 /* ------------------------------------------------------------------------ */
 int64_t orc_padded_k(int64_t K) { return (K + 63) / 64 * 64; }
 int64_t orc_padded_n(int64_t N) { return (N + 7) / 8 * 8; }
@@ -109,18 +112,15 @@ static int64_t orc_code_byte_offset(int64_t n, int64_t k, int64_t K)
 }
 static int orc_code_bit_offset(int64_t k) { return (int)(2 * ((k % 16) / 4)); }
 
-static uint8_t orc_code_to_bits(int8_t c)
-{
-    return c == 0 ? 0u : (c == 1 ? 1u : 2u);   /* [BHFRC] sec. 4.1 table */
-}
+static uint8_t orc_code_to_bits(int8_t c) { return (uint8_t)(c + 1); }   /* -1,0,+1 -> 0,1,2 */
 
 void orc_pack(const int8_t* code, int64_t N, int64_t K, uint8_t* packed)
 {
     const int64_t Np = orc_padded_n(N), Kp = orc_padded_k(K);
-    memset(packed, 0xFF, (size_t)orc_packed_bytes(N, K));   /* all 11 = padding */
+    memset(packed, 0x55, (size_t)orc_packed_bytes(N, K));   /* all 01 = padding */
     for (int64_t n = 0; n < Np; ++n) {
         for (int64_t k = 0; k < Kp; ++k) {
-            uint8_t bits = (n < N && k < K) ? orc_code_to_bits(code[n * K + k]) : 3u;
+            uint8_t bits = (n < N && k < K) ? orc_code_to_bits(code[n * K + k]) : 1u;
             int64_t off = orc_code_byte_offset(n, k, K);
             int sh = orc_code_bit_offset(k);
             packed[off] = (uint8_t)((packed[off] & ~(3u << sh)) | (bits << sh));
@@ -129,7 +129,7 @@ void orc_pack(const int8_t* code, int64_t N, int64_t K, uint8_t* packed)
 }
 
 /* Inverse of orc_pack.  Returns the number of malformed fields found:      */
-/* a real position holding 11, or a padded position not holding 11.         */
+/* any 11, or a padded position not holding 01.                             */
 int64_t orc_unpack(const uint8_t* packed, int64_t N, int64_t K, int8_t* code)
 {
     const int64_t Np = orc_padded_n(N), Kp = orc_padded_k(K);
@@ -140,8 +140,8 @@ int64_t orc_unpack(const uint8_t* packed, int64_t N, int64_t K, int8_t* code)
             unsigned bits = (packed[off] >> orc_code_bit_offset(k)) & 3u;
             if (n < N && k < K) {
                 if (bits == 3u) ++bad;
-                code[n * K + k] = (int8_t)(bits == 1u ? 1 : (bits == 2u ? -1 : 0));
-            } else if (bits != 3u) {
+                code[n * K + k] = (int8_t)((int)bits - 1);
+            } else if (bits != 1u) {
                 ++bad;
             }
         }

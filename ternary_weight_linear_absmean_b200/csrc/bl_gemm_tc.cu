@@ -6,7 +6,8 @@
 // per-token activations.)
 //
 // Persistent kernel, one CTA per SM, looping over 128 (weight rows, MMA M)
-// x 128 (tokens, MMA N) output tiles; K in stages of 128, 8 stages deep.
+// x 128 (tokens, MMA N) output tiles; K in stages of 256 (eight MMAs of
+// K = 32 per barrier round trip), 4 stages deep.
 // The weights never exist as int8 in memory: the packed 2-bit codes are
 // TMA-loaded (4 KiB per stage), eight expansion warps decode them to signed
 // int8 in registers and write them straight into tensor memory with
@@ -15,12 +16,15 @@
 //
 // Tensor memory (512 columns): two 128-column int32 accumulators (tile i is
 // drained by the epilogue while tile i+1 accumulates into the other) and
-// eight 32-column A stages.
+// four 64-column A stages.
 //
 // Warp roles (512 threads):
 //   warp 0       TMEM allocation; TMA producer (one lane)
-//   warp 1       MMA issuer (one lane): 4 x tcgen05.mma (K = 32) per stage,
-//                tcgen05.commit -> stage-free barrier; per tile -> acc-full
+//   warp 1       MMA issuer (one lane): 8 x tcgen05.mma (K = 32) per stage,
+//                tcgen05.commit -> stage-free barrier; per tile -> acc-full.
+//                It waits only for the expansion barrier: the expansion
+//                threads arrive there after observing the stage's TMA
+//                barrier, so the activation tile is complete by then too
 //   warps 4-11   expansion, two groups of four taking alternate stages:
 //                warp w writes TMEM lanes 32*(w%4) .. +31 of its stages
 //   warps 12-15  epilogue: per-token factors gamma32 / s_m (fp64),
@@ -29,11 +33,9 @@
 // All mbarrier waits are bounded (bl_ptx.cuh); every role reaches the final
 // barrier, after which the allocating warp frees the tensor memory.
 //
-// Decode to signed int8: per 2-bit field (lo, hi), code = lo - hi.
-//   S = (w & 0x55555555 | 0xAAAAAAAA) - ((w >> 1) & 0x55555555)
-// holds 2 + code in every field (no borrow between fields; padding 11 -> 2,
-// i.e. code 0).  Field t of every byte, ((S >> 2t) & 0x03030303), plus
-// 0x7E7E7E7E then xor 0x80808080 gives the bytes 0xFF, 0x00, 0x01.
+// Decode to signed int8: the packed fields hold u = code + 1 (include/
+// bitlinear.h); field t of every byte, ((w >> 2t) & 0x03030303), plus
+// 0x7F7F7F7F then xor 0x80808080 gives the bytes 0xFF, 0x00, 0x01.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -45,15 +47,17 @@ namespace {
 
 constexpr int BM = 128;        // weight rows per tile (MMA M)
 constexpr int BN = 128;        // tokens per tile (MMA N)
-constexpr int BK = 128;        // k per stage (bytes of int8)
-constexpr int STAGES = 8;
+constexpr int BK = 256;        // k per stage (bytes of int8): 8 MMAs per barrier round trip
+constexpr int STAGES = 4;
 constexpr int kThreads = 512;
-constexpr int Q_STAGE = BN * BK;             // 16 KiB, 128B-swizzled
-constexpr int W_STAGE = (BM / 8) * 256;      // 16 tiles x 2 chunks x 128 B = 4 KiB
+constexpr int Q_ATOM = BN * 128;             // one 128-byte-wide K slab of the token tile
+constexpr int Q_STAGE = BN * BK;             // 32 KiB: two 128B-swizzled slabs
+constexpr int W_HALF = (BM / 8) * 256;       // 16 tiles x 2 chunks x 128 B = 4 KiB
+constexpr int W_STAGE = 2 * W_HALF;          // 4 chunks of every row: 8 KiB
 constexpr int TMEM_COLS = 512;
 constexpr int ACC_COLS = BN;                 // one accumulator buffer
 constexpr int A_COL0 = 2 * ACC_COLS;         // A stages after the two accumulators
-constexpr int A_STAGE_COLS = BK / 4;         // 32 columns per stage
+constexpr int A_STAGE_COLS = BK / 4;         // 64 columns per stage
 constexpr int EXP_WARP0 = 4, EPI_WARP0 = 12;
 
 struct Smem {
@@ -67,9 +71,12 @@ struct Smem {
     int epi_ok[2];
 };
 
-__device__ __forceinline__ uint32_t signed_codes(int t, uint32_t S)
+// Field t of every byte (u = code + 1 in {0, 1, 2}) -> signed int8 code:
+// u + 0x7F is 0x7F, 0x80 or 0x81 (no carry out of the byte); flipping the
+// top bit gives 0xFF, 0x00, 0x01 = -1, 0, +1.
+__device__ __forceinline__ uint32_t signed_codes(int t, uint32_t w)
 {
-    return (((S >> (2 * t)) & 0x03030303u) + 0x7E7E7E7Eu) ^ 0x80808080u;
+    return (((w >> (2 * t)) & 0x03030303u) + 0x7F7F7F7Fu) ^ 0x80808080u;
 }
 
 __device__ __forceinline__ uint64_t make_bdesc(uint32_t smem_addr)
@@ -198,7 +205,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
                     }
                     mbar_arrive_expect_tx(&sm.full[s], Q_STAGE + W_STAGE);
                     tma_load_2d(sm.q[s], &tmap_q, kb * BK, m0, &sm.full[s]);
-                    tma_load_2d(sm.w[s], &tmap_w, kb * 256, n0 / 8, &sm.full[s]);
+                    tma_load_2d(sm.q[s] + Q_ATOM, &tmap_q, kb * BK + 128, m0, &sm.full[s]);
+                    tma_load_2d(sm.w[s], &tmap_w, kb * 512, n0 / 8, &sm.full[s]);
+                    tma_load_2d(sm.w[s] + W_HALF, &tmap_w, kb * 512 + 256, n0 / 8, &sm.full[s]);
                 }
             }
             // every copy issued has landed before this thread leaves
@@ -218,8 +227,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
                 for (int kb = 0; kb < nk; ++kb, ++g) {
                     const int s = g % STAGES;
                     const uint32_t ph = (g / STAGES) & 1;
-                    if (!wait_parity(&sm.full[s], ph, status, abort) ||
-                        !wait_parity(&sm.expanded[s], ph, status, abort)) {
+                    if (!wait_parity(&sm.expanded[s], ph, status, abort)) {
                         ok = false;
                         break;
                     }
@@ -227,8 +235,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
                     const uint32_t qaddr = smem_u32(sm.q[s]);
 #pragma unroll
                     for (int j = 0; j < BK / 32; ++j)
-                        mma_i8_ts(d_tmem, tmem + A_COL0 + s * A_STAGE_COLS + j * 8, make_bdesc(qaddr + j * 32),
-                                  (kb | j) != 0);
+                        mma_i8_ts(d_tmem, tmem + A_COL0 + s * A_STAGE_COLS + j * 8,
+                                  make_bdesc(qaddr + (j >> 2) * Q_ATOM + (j & 3) * 32), (kb | j) != 0);
                     mma_commit(&sm.empty[s]);
                 }
                 if (ok) mma_commit(&sm.acc_full[b]);
@@ -256,20 +264,21 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
                     ok = false;
                     break;
                 }
-                uint32_t out[32];
 #pragma unroll
-                for (int cl = 0; cl < 2; ++cl) {
-                    const uint4 wv = *reinterpret_cast<const uint4*>(sm.w[s] + woff + cl * 128);
-                    const uint32_t words[4] = {wv.x, wv.y, wv.z, wv.w};
+                for (int h = 0; h < 2; ++h) {          // chunks 2h, 2h+1 of the stage
+                    uint32_t out[32];
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const uint32_t w = words[i];
-                        const uint32_t S = ((w & 0x55555555u) | 0xAAAAAAAAu) - ((w >> 1) & 0x55555555u);
+                    for (int cl = 0; cl < 2; ++cl) {
+                        const uint4 wv = *reinterpret_cast<const uint4*>(sm.w[s] + h * W_HALF + woff + cl * 128);
+                        const uint32_t words[4] = {wv.x, wv.y, wv.z, wv.w};
 #pragma unroll
-                        for (int tt = 0; tt < 4; ++tt) out[16 * cl + 4 * i + tt] = signed_codes(tt, S);
+                        for (int i = 0; i < 4; ++i) {
+#pragma unroll
+                            for (int tt = 0; tt < 4; ++tt) out[16 * cl + 4 * i + tt] = signed_codes(tt, words[i]);
+                        }
                     }
+                    tmem_st32(tmem + lane_base + A_COL0 + s * A_STAGE_COLS + 32 * h, out);
                 }
-                tmem_st32(tmem + lane_base + A_COL0 + s * A_STAGE_COLS, out);
                 tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(&sm.expanded[s]);
@@ -393,7 +402,7 @@ cudaError_t launch_gemm_tc(const int8_t* q, const float* s, const uint8_t* packe
     const int64_t Kp = padded_k(K);
     const int64_t TB = chunks_per_row(K) * 128;
     CUtensorMap tq, tw;
-    if (!make_2d_u8(&tq, q, (uint64_t)Kp, (uint64_t)M, (uint64_t)Kp, BK, BN, CU_TENSOR_MAP_SWIZZLE_128B))
+    if (!make_2d_u8(&tq, q, (uint64_t)Kp, (uint64_t)M, (uint64_t)Kp, 128, BN, CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
     if (!make_2d_u8(&tw, packed, (uint64_t)TB, (uint64_t)(padded_n(N) / 8), (uint64_t)TB, 256, BM / 8,
                     CU_TENSOR_MAP_SWIZZLE_NONE))

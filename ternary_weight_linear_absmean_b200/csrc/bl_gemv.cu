@@ -10,16 +10,12 @@
 // [16l, 16l+16) of the span -- one fully coalesced 128-bit load per lane.
 // Lane l works on row r = l % 8 and chunk 4g + l / 8.
 //
-// Decode.  A 32-bit word holds 16 codes (byte b, field t -> k = 16i+4t+b).
-// With lo/hi the two bits of a field, u = 1 + lo - hi is 1 + code in {0,1,2}
-// (11 padding -> 1, i.e. code 0).  For all 16 fields at once:
-//     U = (w & 0x55555555) + 0x55555555 - ((w >> 1) & 0x55555555)
-// never carries or borrows between fields.  Field t of every byte is then
-// U & (0x03030303 << 2t), i.e. 4^t * u (for t = 3 taken as (U >> 2) &
-// 0x30303030 = 16 * u, so every byte fits a signed int8); a signed dp4a with
-// the 4 activations k = 16i+4t .. +3 gives f_t * sum(u * q), accumulated in
-// its own register a_t (f = 1, 4, 16, 16).  Finally
-//     sum(code*q) = a_0 + a_1/4 + a_2/16 + a_3/16 - sum_k q_k
+// Decode.  A 32-bit word holds 16 codes (byte b, field t -> k = 16i+4t+b),
+// each stored as u = code + 1 in {0, 1, 2} (padding 01 -> u = 1, code 0).
+// Field t of every byte is w & (0x03030303 << 2t), i.e. 4^t * u; dp4a
+// (unsigned x signed) with the 4 activations k = 16i+4t .. +3 gives
+// 4^t * sum(u * q), accumulated in its own register a_t.  Finally
+//     sum(code*q) = sum_t a_t / 4^t  -  sum_k q_k
 // (all exact integer arithmetic; the shifts divide exact multiples).
 //
 // Epilogue: per-lane totals are reduced over the 4 lanes of a row (shuffle)
@@ -37,11 +33,6 @@ namespace {
 
 constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
-
-__device__ __forceinline__ uint32_t biased_codes(uint32_t w)
-{
-    return (w & 0x55555555u) + 0x55555555u - ((w >> 1) & 0x55555555u);
-}
 
 __device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c)
 {
@@ -203,8 +194,7 @@ gemv_kernel(const __grid_constant__ Batch<G> b, unsigned* status)
             const int c = 4 * g + sub;
             if (c < C) {
                 const uint4 wv = ldg_stream(tile_ptr + (int64_t)g * 512 + lane * 16);
-                const uint32_t U[4] = {biased_codes(wv.x), biased_codes(wv.y), biased_codes(wv.z),
-                                       biased_codes(wv.w)};
+                const uint32_t U[4] = {wv.x, wv.y, wv.z, wv.w};   // stored fields are u = code + 1
 #pragma unroll
                 for (int m = 0; m < MT; ++m) {
                     if (m < mcount) {
@@ -218,10 +208,10 @@ gemv_kernel(const __grid_constant__ Batch<G> b, unsigned* status)
                             uint4 a;
                             if constexpr (FUSED) a = arow[i];
                             else a = __ldg(arow + i);
-                            acc[m][0] = dp4a_ss(U[i] & 0x03030303u, a.x, acc[m][0]);
-                            acc[m][1] = dp4a_ss(U[i] & 0x0C0C0C0Cu, a.y, acc[m][1]);
-                            acc[m][2] = dp4a_ss(U[i] & 0x30303030u, a.z, acc[m][2]);
-                            acc[m][3] = dp4a_ss((U[i] >> 2) & 0x30303030u, a.w, acc[m][3]);
+                            acc[m][0] = dp4a_us(U[i] & 0x03030303u, a.x, acc[m][0]);
+                            acc[m][1] = dp4a_us(U[i] & 0x0C0C0C0Cu, a.y, acc[m][1]);
+                            acc[m][2] = dp4a_us(U[i] & 0x30303030u, a.z, acc[m][2]);
+                            acc[m][3] = dp4a_us(U[i] & 0xC0C0C0C0u, a.w, acc[m][3]);
                         }
                     }
                 }
@@ -231,7 +221,7 @@ gemv_kernel(const __grid_constant__ Batch<G> b, unsigned* status)
         // ---- reduce: fields, 4 lanes of a row, 8 warps
 #pragma unroll
         for (int m = 0; m < MT; ++m) {
-            int tot = acc[m][0] + (acc[m][1] >> 2) + (acc[m][2] >> 4) + (acc[m][3] >> 4);
+            int tot = acc[m][0] + (acc[m][1] >> 2) + (acc[m][2] >> 4) + (acc[m][3] >> 6);
             tot += __shfl_xor_sync(0xffffffffu, tot, 8);
             tot += __shfl_xor_sync(0xffffffffu, tot, 16);
             if (sub == 0) red[warp][m][r] = tot;

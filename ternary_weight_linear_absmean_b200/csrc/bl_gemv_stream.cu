@@ -17,8 +17,8 @@
 //                   form) or copy q there, while the first stages are in
 //                   flight; then for each stage take 512-byte spans (4 chunks
 //                   x 8 rows of a tile) round-robin, lane l reading 16 bytes,
-//                   row r = l % 8, and accumulate with signed dp4a (decode
-//                   as in bl_gemv.cu).  Per-lane partial sums are added into a
+//                   row r = l % 8, and accumulate with dp4a (decode as in
+//                   bl_gemv.cu).  Per-lane partial sums are added into a
 //                   per-(tile, row, token) int32 array in shared memory
 //                   (integer adds: exact and order-independent) whenever the
 //                   lane's tile changes.
@@ -184,7 +184,7 @@ __device__ float quantise_row(const XT* __restrict__ row, int K, int Kp, int8_t*
 template <int MT>
 __device__ __forceinline__ void dot_chunk(const uint4 wv, const int8_t* qs, int Kp, int c, int (&acc)[MT][4])
 {
-    const uint32_t U[4] = {biased_codes(wv.x), biased_codes(wv.y), biased_codes(wv.z), biased_codes(wv.w)};
+    const uint32_t U[4] = {wv.x, wv.y, wv.z, wv.w};   // stored fields are u = code + 1
 #pragma unroll
     for (int m = 0; m < MT; ++m) {
         {
@@ -192,10 +192,10 @@ __device__ __forceinline__ void dot_chunk(const uint4 wv, const int8_t* qs, int 
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const uint4 a = a4[i];
-                acc[m][0] = dp4a_ss(U[i] & 0x03030303u, a.x, acc[m][0]);
-                acc[m][1] = dp4a_ss(U[i] & 0x0C0C0C0Cu, a.y, acc[m][1]);
-                acc[m][2] = dp4a_ss(U[i] & 0x30303030u, a.z, acc[m][2]);
-                acc[m][3] = dp4a_ss((U[i] >> 2) & 0x30303030u, a.w, acc[m][3]);
+                acc[m][0] = dp4a_us(U[i] & 0x03030303u, a.x, acc[m][0]);
+                acc[m][1] = dp4a_us(U[i] & 0x0C0C0C0Cu, a.y, acc[m][1]);
+                acc[m][2] = dp4a_us(U[i] & 0x30303030u, a.z, acc[m][2]);
+                acc[m][3] = dp4a_us(U[i] & 0xC0C0C0C0u, a.w, acc[m][3]);
             }
         }
     }
@@ -327,7 +327,7 @@ stream_kernel(const __grid_constant__ StreamBatch b, unsigned* status)
 #pragma unroll
             for (int m = 0; m < MT; ++m) {
                 if (m < M) {
-                    const int tot = acc[m][0] + (acc[m][1] >> 2) + (acc[m][2] >> 4) + (acc[m][3] >> 4);
+                    const int tot = acc[m][0] + (acc[m][1] >> 2) + (acc[m][2] >> 4) + (acc[m][3] >> 6);
                     atomicAdd(&sacc[(cur * 8 + r) * MT + m], tot);
                 }
 #pragma unroll

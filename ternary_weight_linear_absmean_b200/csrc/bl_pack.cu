@@ -1,7 +1,8 @@
 // bl_pack.cu -- absmean ternary quantisation of a weight tensor and the
 // 2-bit packed layout (BitNet b1.58, aratech.ae "Ternary weights {-1, 0, +1}":
-// scale = 1/mean|W|, W_q = clip(-1, 1)(round(W * scale)); code values from
-// bhfrc.com/news/56965 sec. 4.1).
+// scale = 1/mean|W|, W_q = clip(-1, 1)(round(W * scale)); 2 bits per weight
+// as in bhfrc.com/news/56965 sec. 4.1, stored as code + 1 -- see
+// include/bitlinear.h).
 //
 // Three launches, all HBM-bound streaming passes:
 //   1. absmean_partial: each block sums |W| over a fixed grid-stride slice
@@ -94,10 +95,10 @@ absmean_finalize_kernel(const double* __restrict__ partial, int blocks, int64_t 
     }
 }
 
-// 2-bit value of one weight: 01 for +1, 10 for -1, 00 for 0.
+// 2-bit value of one weight, code + 1: 10 for +1, 01 for 0, 00 for -1.
 __device__ __forceinline__ uint32_t code_bits(float w, float thr)
 {
-    return (w > thr) ? 1u : ((w < -thr) ? 2u : 0u);
+    return (w > thr) ? 2u : ((w < -thr) ? 0u : 1u);
 }
 
 __global__ void __launch_bounds__(256)
@@ -114,7 +115,7 @@ pack_kernel(const float* __restrict__ W, int64_t N, int64_t K, int64_t total,
     const int64_t n = tile * 8 + r;
     uint4 out;
     if (n >= N) {
-        out = make_uint4(0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu);
+        out = make_uint4(0x55555555u, 0x55555555u, 0x55555555u, 0x55555555u);   // padding rows: 01
     } else {
         const float thr = *thr_p;
         const float* row = W + n * K;
@@ -144,7 +145,7 @@ pack_kernel(const float* __restrict__ W, int64_t N, int64_t K, int64_t total,
                 for (int f = 0; f < 4; ++f)
                     for (int b = 0; b < 4; ++b) {
                         const int64_t k = k0 + 16 * i + 4 * f + b;
-                        const uint32_t bits = (k < K) ? code_bits(row[k], thr) : 3u;
+                        const uint32_t bits = (k < K) ? code_bits(row[k], thr) : 1u;
                         w |= bits << (8 * b + 2 * f);
                     }
                 word[i] = w;

@@ -145,11 +145,4 @@ __device__ __forceinline__ int dp4a_ss(uint32_t a, uint32_t b, int c)
     return d;
 }
 
-// 16 ternary codes of one packed word -> 1 + code (0, 1 or 2) per 2-bit
-// field, in place: (lo + 1 - hi) per field never carries between fields.
-__device__ __forceinline__ uint32_t biased_codes(uint32_t w)
-{
-    return (w & 0x55555555u) + 0x55555555u - ((w >> 1) & 0x55555555u);
-}
-
 }  // namespace bl

@@ -154,41 +154,43 @@ def _hexbytes(s):
 
 
 def test_pack_all_plus_one_and_all_minus_one():
-    # N=1, K=64 -> 8 padded rows x 1 chunk = 128 bytes.  Row 0 is bytes 0..15;
-    # code +1 = 01 in all four fields of a byte -> 0x55; -1 = 10 -> 0xAA.
-    # Padded rows 1..7 are all 11 -> 0xFF.
+    # The layout stores u = code + 1 (include/bitlinear.h): +1 -> 10, 0 -> 01,
+    # -1 -> 00, padding 01.  N=1, K=64 -> 8 padded rows x 1 chunk = 128 bytes.
+    # Row 0 is bytes 0..15: all +1 -> 0b10101010 = 0xAA; all -1 -> 0x00.
+    # Padded rows 1..7 are all 01 -> 0x55.
     plus = oracle.pack(np.ones((1, 64), np.int8))
     minus = oracle.pack(-np.ones((1, 64), np.int8))
-    assert np.array_equal(plus, _hexbytes("55" * 16 + "ff" * 112))
-    assert np.array_equal(minus, _hexbytes("aa" * 16 + "ff" * 112))
+    assert np.array_equal(plus, _hexbytes("aa" * 16 + "55" * 112))
+    assert np.array_equal(minus, _hexbytes("00" * 16 + "55" * 112))
 
 
 def test_pack_single_code_position():
-    # k = 45 = 16*2 + 4*3 + 1 -> word 2, field 3, byte 1 -> byte offset
-    # 2*4 + 1 = 9, bits 6..7 -> 0x40.
+    # Zero codes are 01 -> bytes 0x55.  k = 45 = 16*2 + 4*3 + 1 -> word 2,
+    # field 3, byte 1 -> byte offset 2*4 + 1 = 9, bits 6..7:
+    #   +1 (10): 0b10_01_01_01 = 0x95;  -1 (00): 0b00_01_01_01 = 0x15.
     code = np.zeros((1, 64), np.int8)
     code[0, 45] = 1
-    assert np.array_equal(oracle.pack(code), _hexbytes("00" * 9 + "40" + "00" * 6 + "ff" * 112))
+    assert np.array_equal(oracle.pack(code), _hexbytes("55" * 9 + "95" + "55" * 6 + "55" * 112))
     code[0, 45] = -1
-    assert np.array_equal(oracle.pack(code), _hexbytes("00" * 9 + "80" + "00" * 6 + "ff" * 112))
+    assert np.array_equal(oracle.pack(code), _hexbytes("55" * 9 + "15" + "55" * 6 + "55" * 112))
 
 
 def test_pack_ragged_tile_and_chunk():
     # N=9, K=70 -> Np=16, Kp=128, C=2, 512 bytes.  Row 8 is row 0 of tile 1
     # (tile stride 8*2*16 = 256).  k = 69: chunk 1, word 0, field 1, byte 1
     # -> offset 256 + (1*8 + 0)*16 + 1 = 385.  That byte's fields cover
-    # k = 65 (code 0 -> 00), 69 (+1 -> 01), 73 and 77 (padding -> 11):
-    # 0b11_11_01_00 = 0xF4.
+    # k = 65 (code 0 -> 01), 69 (+1 -> 10), 73 and 77 (padding -> 01):
+    # 0b01_01_10_01 = 0x59.
     code = np.zeros((9, 70), np.int8)
     code[8, 69] = 1
     p = oracle.pack(code)
     assert p.size == 512
-    assert p[385] == 0xF4
+    assert p[385] == 0x59
     # Row 9 (tile 1, r = 1) is padding: offsets 256 + (c*8 + 1)*16 .. +16.
     for c in range(2):
-        assert np.all(p[256 + (c * 8 + 1) * 16: 256 + (c * 8 + 2) * 16] == 0xFF)
+        assert np.all(p[256 + (c * 8 + 1) * 16: 256 + (c * 8 + 2) * 16] == 0x55)
     # Row 0, chunk 0 (offset 0..15) is a full chunk of zero codes.
-    assert np.all(p[0:16] == 0)
+    assert np.all(p[0:16] == 0x55)
 
 
 @pytest.mark.parametrize("N,K", [(1, 1), (3, 64), (8, 65), (13, 200), (64, 256)])
