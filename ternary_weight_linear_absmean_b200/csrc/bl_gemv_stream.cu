@@ -108,24 +108,37 @@ __device__ float quantise_row(const XT* __restrict__ row, int K, int Kp, int8_t*
     const int t = threadIdx.x - 32;
     constexpr bool BF16 = sizeof(XT) == 2;
     constexpr int VE = 16 / sizeof(XT);   // elements per 16-byte vector
+    constexpr int VR = 4;                 // vectors a thread keeps in registers
+    const int nv = K / VE;
     const bool vec = (K % VE) == 0;
+    const bool held = vec && nv <= VR * kConsumers;   // pass 2 needs no reload
+    uint4 keep[VR];
     uint32_t mbits = 0;                   // max |x| bit pattern (fp32 layout)
-    if (vec) {
-        const uint4* rv = reinterpret_cast<const uint4*>(row);
-        uint32_t mhi = 0, mlo = 0;
-        for (int v = t; v < K / VE; v += kConsumers) {
-            const uint4 u = __ldg(rv + v);
-            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+    uint32_t mhi = 0, mlo = 0;
+    auto amax_of = [&](const uint4 u) {
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                if constexpr (BF16) {
-                    mhi = max(mhi, w[i] & 0x7FFF0000u);
-                    mlo = max(mlo, (w[i] << 16) & 0x7FFF0000u);
-                } else {
-                    mhi = max(mhi, w[i] & 0x7FFFFFFFu);
-                }
+        for (int i = 0; i < 4; ++i) {
+            if constexpr (BF16) {
+                mhi = max(mhi, w[i] & 0x7FFF0000u);
+                mlo = max(mlo, (w[i] << 16) & 0x7FFF0000u);
+            } else {
+                mhi = max(mhi, w[i] & 0x7FFFFFFFu);
             }
         }
+    };
+    const uint4* rv = reinterpret_cast<const uint4*>(row);
+    if (held) {
+#pragma unroll
+        for (int j = 0; j < VR; ++j) {
+            const int v = t + j * kConsumers;
+            keep[j] = v < nv ? __ldg(rv + v) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int j = 0; j < VR; ++j) amax_of(keep[j]);   // zero padding does not change the max
+        mbits = max(mhi, mlo);
+    } else if (vec) {
+        for (int v = t; v < nv; v += kConsumers) amax_of(__ldg(rv + v));
         mbits = max(mhi, mlo);
     } else {
         for (int k = t; k < K; k += kConsumers) mbits = max(mbits, __float_as_uint(to_f(row[k])) & 0x7FFFFFFFu);
@@ -135,31 +148,38 @@ __device__ float quantise_row(const XT* __restrict__ row, int K, int Kp, int8_t*
     const float amax = fmaxf(__uint_as_float(mbits), 1e-5f);
     const float s = 127.0f / amax;
     int part = 0;
-    if (vec) {
-        const uint4* rv = reinterpret_cast<const uint4*>(row);
-        for (int v = t; v < K / VE; v += kConsumers) {
-            const uint4 u = __ldg(rv + v);
-            if constexpr (BF16) {
-                const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-                int c[8];
+    auto quant_store = [&](const uint4 u, int v) {
+        if constexpr (BF16) {
+            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+            int c[8];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    c[2 * i] = __float2int_rn(__fmul_rn(__uint_as_float(w[i] << 16), s));
-                    c[2 * i + 1] = __float2int_rn(__fmul_rn(__uint_as_float(w[i] & 0xFFFF0000u), s));
-                }
-                const uint32_t p0 = pack4(c[0], c[1], c[2], c[3]);
-                const uint32_t p1 = pack4(c[4], c[5], c[6], c[7]);
-                part = dp4a_ss(p0, 0x01010101u, part);
-                part = dp4a_ss(p1, 0x01010101u, part);
-                *reinterpret_cast<uint2*>(q + v * 8) = make_uint2(p0, p1);
-            } else {
-                const uint32_t p0 = pack4(__float2int_rn(__fmul_rn(__uint_as_float(u.x), s)),
-                                          __float2int_rn(__fmul_rn(__uint_as_float(u.y), s)),
-                                          __float2int_rn(__fmul_rn(__uint_as_float(u.z), s)),
-                                          __float2int_rn(__fmul_rn(__uint_as_float(u.w), s)));
-                part = dp4a_ss(p0, 0x01010101u, part);
-                *reinterpret_cast<uint32_t*>(q + v * 4) = p0;
+            for (int i = 0; i < 4; ++i) {
+                c[2 * i] = __float2int_rn(__fmul_rn(__uint_as_float(w[i] << 16), s));
+                c[2 * i + 1] = __float2int_rn(__fmul_rn(__uint_as_float(w[i] & 0xFFFF0000u), s));
             }
+            const uint32_t p0 = pack4(c[0], c[1], c[2], c[3]);
+            const uint32_t p1 = pack4(c[4], c[5], c[6], c[7]);
+            part = dp4a_ss(p0, 0x01010101u, part);
+            part = dp4a_ss(p1, 0x01010101u, part);
+            *reinterpret_cast<uint2*>(q + v * 8) = make_uint2(p0, p1);
+        } else {
+            const uint32_t p0 = pack4(__float2int_rn(__fmul_rn(__uint_as_float(u.x), s)),
+                                      __float2int_rn(__fmul_rn(__uint_as_float(u.y), s)),
+                                      __float2int_rn(__fmul_rn(__uint_as_float(u.z), s)),
+                                      __float2int_rn(__fmul_rn(__uint_as_float(u.w), s)));
+            part = dp4a_ss(p0, 0x01010101u, part);
+            *reinterpret_cast<uint32_t*>(q + v * 4) = p0;
+        }
+    };
+    if (vec) {
+        if (held) {
+#pragma unroll
+            for (int j = 0; j < VR; ++j) {
+                const int v = t + j * kConsumers;
+                if (v < nv) quant_store(keep[j], v);
+            }
+        } else {
+            for (int v = t; v < nv; v += kConsumers) quant_store(__ldg(rv + v), v);
         }
         for (int k4 = K + 4 * t; k4 < Kp; k4 += 4 * kConsumers) *reinterpret_cast<uint32_t*>(q + k4) = 0u;
     } else {
@@ -214,19 +234,20 @@ stream_kernel(const __grid_constant__ StreamBatch b, unsigned* status)
     __shared__ int abort_flag;
     __shared__ int piece_ok[2];
 
-    // ---- which problem, which tiles
+    // ---- which problem, which tiles (cheap: the CTA's first copy waits on it)
     int pi = 0;
 #pragma unroll 1
     for (int i = 1; i < b.count; ++i)
-        if ((int)blockIdx.x >= b.p[i].cta_begin) pi = i;
+        if ((int)blockIdx.x >= b.cta_begin[i]) pi = i;
     const StreamProblem& P = b.p[pi];
     const int K = (int)P.K, Kp = (int)padded_k(P.K);
     const int64_t N = P.N;
     const uint32_t TB = (uint32_t)(chunks_per_row(K) * 128);   // bytes per tile
-    const int64_t tiles = padded_n(N) / 8;
-    const int64_t ci = (int64_t)blockIdx.x - P.cta_begin;
-    const int64_t t0 = tiles * ci / P.ctas, t1 = tiles * (ci + 1) / P.ctas;
-    const uint32_t range = (uint32_t)((t1 - t0) * TB);            // < 2^31 (host-checked)
+    const int ci = (int)blockIdx.x - P.cta_begin;
+    const int64_t t0 = (int64_t)ci * P.tiles_base + (ci < P.tiles_extra ? ci : P.tiles_extra);
+    const int ntl = P.tiles_base + (ci < P.tiles_extra ? 1 : 0);
+    const int64_t t1 = t0 + ntl;
+    const uint32_t range = (uint32_t)ntl * TB;                    // < 2^31 (host-checked)
     const uint8_t* src = P.packed + t0 * (int64_t)TB;
     const int stages = b.stages;
     const int npieces = (int)((range + kStageBytes - 1) / kStageBytes);
@@ -236,6 +257,13 @@ stream_kernel(const __grid_constant__ StreamBatch b, unsigned* status)
     int* sacc = reinterpret_cast<int*>(smem + (size_t)stages * kStageBytes + b.q_bytes);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // The producer initialises the barriers and puts the first `stages`
+    // pieces in flight straight away; the consumers quantise x meanwhile and
+    // the whole CTA meets at the __syncthreads below before anyone waits.
+    const int first = npieces < stages ? npieces : stages;
+    // Let the next kernel in the stream start launching now; it waits for
+    // this one to finish before it touches anything this one writes.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if (threadIdx.x == 0) {
         for (int s = 0; s < stages; ++s) {
             mbar_init(&full_bar[s], 1);
@@ -243,16 +271,77 @@ stream_kernel(const __grid_constant__ StreamBatch b, unsigned* status)
         }
         abort_flag = 0;
         fence_barrier_init();
+        // This grid may have started before the previous kernel finished
+        // (programmatic dependent launch), so nothing it reads is safe to
+        // read yet -- but an L2 prefetch is: it only warms the coherent L2,
+        // and the copies below read after the wait.  Only the bytes of the
+        // first copies: more would just evict each other on large layers.
+        const uint32_t head = (uint32_t)first * kStageBytes < range ? (uint32_t)first * kStageBytes : range;
+        for (uint32_t o = 0; o < head; o += kStageBytes)
+            prefetch_l2_bulk(src + o, (head - o) < (uint32_t)kStageBytes ? (head - o) : (uint32_t)kStageBytes);
+    }
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (threadIdx.x == 0) {
+        for (int j = 0; j < first; ++j) {
+            const uint32_t left = range - (uint32_t)j * kStageBytes;
+            const uint32_t len = left < (uint32_t)kStageBytes ? left : (uint32_t)kStageBytes;
+            mbar_arrive_expect_tx(&full_bar[j], len);
+            bulk_g2s(ring + (size_t)j * kStageBytes, src + (int64_t)j * kStageBytes, len, &full_bar[j]);
+        }
+    }
+
+    const int M = b.M;
+    if (warp != 0) {
+        // ------------------------------------------- consumers: prologue
+        for (int i = threadIdx.x - 32; i < ntl * 8 * MT; i += kConsumers) sacc[i] = 0;
+        if constexpr (FUSED) {
+            const XT* xb = static_cast<const XT*>(P.x);
+#pragma unroll 1
+            for (int m = 0; m < M; ++m) {
+                int sq;
+                const float s = quantise_row<XT>(xb + (int64_t)m * K, K, Kp, qs + m * Kp, redi, &sq, status);
+                if (threadIdx.x == 32) {
+                    s_scale[m] = s;
+                    s_sumq[m] = sq;
+                }
+                named_bar(1, kConsumers);
+            }
+        } else {
+#pragma unroll 1
+            for (int m = 0; m < M; ++m) {
+                const uint4* gq = reinterpret_cast<const uint4*>(P.q + (int64_t)m * Kp);
+                uint4* sq4 = reinterpret_cast<uint4*>(qs + m * Kp);
+                int part = 0;
+                for (int v = threadIdx.x - 32; v < Kp / 16; v += kConsumers) {
+                    const uint4 u = __ldg(gq + v);
+                    sq4[v] = u;
+                    part = dp4a_ss(u.x, 0x01010101u, part);
+                    part = dp4a_ss(u.y, 0x01010101u, part);
+                    part = dp4a_ss(u.z, 0x01010101u, part);
+                    part = dp4a_ss(u.w, 0x01010101u, part);
+                }
+                const int sq = consumers_sum(part, redi);
+                if (threadIdx.x == 32) {
+                    s_scale[m] = P.s[m];
+                    s_sumq[m] = sq;
+                }
+                named_bar(1, kConsumers);
+            }
+        }
+        // token slots M .. MT-1 get zero activations, so the dot loop needs
+        // no token guard (their sums are never written out)
+        for (int i = threadIdx.x - 32; i < (MT - M) * Kp / 16; i += kConsumers)
+            reinterpret_cast<uint4*>(qs + M * Kp)[i] = make_uint4(0, 0, 0, 0);
     }
     __syncthreads();
 
     if (warp == 0) {
         // ------------------------------------------------------ producer
         if (lane == 0) {
-            int issued = 0;
-            for (int j = 0; j < npieces; ++j) {
+            int issued = first;
+            for (int j = first; j < npieces; ++j) {
                 const int s = j % stages, round = j / stages;
-                if (round > 0 && !wait_parity(&empty_bar[s], (round - 1) & 1, status, &abort_flag)) break;
+                if (!wait_parity(&empty_bar[s], (round - 1) & 1, status, &abort_flag)) break;
                 const uint32_t left = range - (uint32_t)j * kStageBytes;
                 const uint32_t len = left < (uint32_t)kStageBytes ? left : (uint32_t)kStageBytes;
                 mbar_arrive_expect_tx(&full_bar[s], len);
@@ -262,56 +351,13 @@ stream_kernel(const __grid_constant__ StreamBatch b, unsigned* status)
             // every copy this thread issued lands before it exits (the last
             // use of each stage is that stage's latest phase)
             for (int j = issued - stages < 0 ? 0 : issued - stages; j < issued; ++j)
-                wait_parity(&full_bar[j % stages], (j / stages) & 1, status, nullptr);
+                wait_parity(&full_bar[j % stages], (j / stages) & 1, status, nullptr, true);
         }
         return;
     }
 
-    // ---------------------------------------------------------- consumers
+    // ---------------------------------------------------- consumers: loop
     const int cw = warp - 1;
-    const int M = b.M;
-    const int ntl = (int)(t1 - t0);
-    for (int i = threadIdx.x - 32; i < ntl * 8 * MT; i += kConsumers) sacc[i] = 0;
-    if constexpr (FUSED) {
-        const XT* xb = static_cast<const XT*>(P.x);
-#pragma unroll 1
-        for (int m = 0; m < M; ++m) {
-            int sq;
-            const float s = quantise_row<XT>(xb + (int64_t)m * K, K, Kp, qs + m * Kp, redi, &sq, status);
-            if (threadIdx.x == 32) {
-                s_scale[m] = s;
-                s_sumq[m] = sq;
-            }
-            named_bar(1, kConsumers);
-        }
-    } else {
-#pragma unroll 1
-        for (int m = 0; m < M; ++m) {
-            const uint4* gq = reinterpret_cast<const uint4*>(P.q + (int64_t)m * Kp);
-            uint4* sq4 = reinterpret_cast<uint4*>(qs + m * Kp);
-            int part = 0;
-            for (int v = threadIdx.x - 32; v < Kp / 16; v += kConsumers) {
-                const uint4 u = __ldg(gq + v);
-                sq4[v] = u;
-                part = dp4a_ss(u.x, 0x01010101u, part);
-                part = dp4a_ss(u.y, 0x01010101u, part);
-                part = dp4a_ss(u.z, 0x01010101u, part);
-                part = dp4a_ss(u.w, 0x01010101u, part);
-            }
-            const int sq = consumers_sum(part, redi);
-            if (threadIdx.x == 32) {
-                s_scale[m] = P.s[m];
-                s_sumq[m] = sq;
-            }
-            named_bar(1, kConsumers);
-        }
-    }
-
-    // token slots M .. MT-1 get zero activations, so the dot loop needs no
-    // token guard (their sums are never written out)
-    for (int i = threadIdx.x - 32; i < (MT - M) * Kp / 16; i += kConsumers)
-        reinterpret_cast<uint4*>(qs + M * Kp)[i] = make_uint4(0, 0, 0, 0);
-    named_bar(1, kConsumers);
 
     const int r = lane & 7;
     const int sub = lane >> 3;
@@ -446,7 +492,23 @@ cudaError_t launch_t(const StreamBatch& b, int grid, size_t smem, unsigned* stat
         if (e != cudaSuccess) return e;
         configured[dev] = true;
     }
-    fn<<<grid, kThreads, smem, st>>>(b, status);
+    // Programmatic dependent launch: this grid may start while the previous
+    // kernel in the stream is still finishing.  Until griddepcontrol.wait it
+    // only sets up and prefetches its weights into L2; every read of an
+    // input and every write happens after the wait, so a dependency on the
+    // previous kernel (e.g. the packer that wrote the weights) stays safe.
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, fn, b, status);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
@@ -535,6 +597,9 @@ bool plan_stream(StreamBatch& b, int minb, int* grid, size_t* smem)
         const int64_t tiles = padded_n(b.p[i].N) / 8;
         if (b.p[i].ctas > tiles) b.p[i].ctas = (int)tiles;
         b.p[i].cta_begin = begin;
+        b.cta_begin[i] = begin;
+        b.p[i].tiles_base = (int)(tiles / b.p[i].ctas);
+        b.p[i].tiles_extra = (int)(tiles % b.p[i].ctas);
         begin += b.p[i].ctas;
         const int64_t per = (tiles + b.p[i].ctas - 1) / b.p[i].ctas;
         tiles_max = tiles_max > per ? tiles_max : per;

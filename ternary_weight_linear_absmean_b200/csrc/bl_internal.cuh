@@ -80,8 +80,11 @@ struct StreamProblem {
     int64_t N, K;
     int cta_begin;          // set by plan_stream
     int ctas;               // set by plan_stream
+    int tiles_base;         // set by plan_stream: every CTA gets tiles_base tiles,
+    int tiles_extra;        //   the first tiles_extra CTAs one more
 };
 struct StreamBatch {
+    int cta_begin[kMaxGroup];   // copy of p[i].cta_begin, packed for the CTA -> problem search
     StreamProblem p[kMaxGroup];
     int count;
     int M;
