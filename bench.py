@@ -55,6 +55,8 @@ def parse_args():
     ap.add_argument("--mode", choices=["grouped", "fused", "separate"], default="grouped",
                     help="decode: grouped = one launch per step; fused = one launch per linear; "
                          "separate = quantise + product launches per linear")
+    ap.add_argument("--decode-kernel", choices=["auto", "tensor", "dp4a", "tile"], default="auto",
+                    help="decode kernel for M <= 16 (bitlinear_set_decode_kernel)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="oracle CPU-baseline budget")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -133,6 +135,26 @@ class ClockSampler:
 def decode_bytes(lin, M):
     """Algorithmic bytes of one decode pass: packed W + bf16 x + fp32 y."""
     return sum(L["N"] * L["K"] // 4 + M * L["K"] * 2 + M * L["N"] * 4 for L in lin)
+
+
+# DRAM bytes (read + write) per launch of the dominant kernel, from one ncu
+# capture of the same launch configuration (profiles/ holds the summary and
+# the command).  Valid only for the kernel source it was taken from: set an
+# entry to None when that kernel changes.
+MEASURED_TRAFFIC = {
+    # stream_kernel<1, fused, bf16, fp32, 4>, 2B block, M = 1, grouped launch
+    ("block2b", "stream_kernel", 1): 17_463_552,
+}
+
+
+def decode_kernel_name(args, M=1):
+    """The kernel bitlinear_set_decode_kernel selects for the bench shapes:
+    AUTO takes the dp4a streaming kernel up to 4 tokens, the tensor-core
+    kernel above (both fit every bench shape except where noted by the
+    library's fallbacks)."""
+    if args.decode_kernel == "auto":
+        return "stream_kernel" if M <= 4 else "dec_tc_kernel"
+    return {"tensor": "dec_tc_kernel", "dp4a": "stream_kernel", "tile": "gemv_kernel"}[args.decode_kernel]
 
 
 def max_over_ranks(ms, dist, dev):
@@ -353,7 +375,7 @@ def run_decode(torch, bl, args, lin, M, dev, stream, dist, l2):
 
     # dominant kernel: the product kernel (the whole step in grouped mode)
     if mode == "grouped":
-        kern_ms, kern_bytes, kname = ms / args.steps, nbytes, "stream_kernel (fused quantise, 7 linears, 1 launch)"
+        kern_ms, kern_bytes, kname = ms / args.steps, nbytes, f"{decode_kernel_name(args, M)} (fused quantise, {len(lin)} linears, 1 launch)"
     else:
         def kstep(i):
             c = i % copies
@@ -370,7 +392,7 @@ def run_decode(torch, bl, args, lin, M, dev, stream, dist, l2):
         kms = time_region(torch, stream, lambda: GK.run(reps), dist, dev)
         kern_ms = kms / (reps * len(lin))
         kern_bytes = nbytes / len(lin)
-        kname = "stream_kernel (product, one launch per linear)"
+        kname = f"{decode_kernel_name(args, M)} (product, one launch per linear)"
     return dict(S=S, mode=mode, ms=ms, launches=launches, clocks=clocks, nbytes=nbytes,
                 kern_ms=kern_ms, kern_bytes=kern_bytes, kname=kname)
 
@@ -586,6 +608,9 @@ def main():
     from ternary_weight_linear_absmean_b200 import _build
     _build.build()
     torch.cuda.set_device(local)
+    bl.bitlinear_set_decode_kernel({"auto": bl.BL_DECODE_AUTO, "tensor": bl.BL_DECODE_TENSOR,
+                                    "dp4a": bl.BL_DECODE_DP4A, "tile": bl.BL_DECODE_TILE}[args.decode_kernel])
+    config["decode_kernel"] = args.decode_kernel
     dist = None
     if world > 1:
         import datetime
@@ -625,7 +650,7 @@ def main():
                           "l2_policy": "inputs larger than L2 (17.1 GB resident, streamed once per step)"},
                "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                             "frac": achieved / peaks["hbm_gbs"], "traffic": None,
-                            "kernel": "stream_kernel (80 grouped launches per step)",
+                            "kernel": f"{decode_kernel_name(args, 1)} (80 grouped launches per step)",
                             "avg_launch_us": per_step / R["launches"] * 1e3},
                "gpu_launches": R["launches"] * R["steps"], "clocks": R["clocks"]}
     elif args.workload == "pack":
@@ -650,7 +675,10 @@ def main():
                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int32",
                "data": "synthetic", "config": config,
                "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                            "frac": achieved / peaks["hbm_gbs"], "traffic": None, "kernel": R["kname"],
+                            "frac": achieved / peaks["hbm_gbs"],
+                            "traffic": (MEASURED_TRAFFIC.get((args.workload, decode_kernel_name(args, M), M))
+                                        if R["mode"] == "grouped" else None),
+                            "kernel": R["kname"],
                             "peak_kind": f"{peaks['kind']} HBM copy bandwidth (burst)",
                             "algorithmic_bytes_per_launch": R["kern_bytes"],
                             "avg_launch_us": R["kern_ms"] * 1e3},

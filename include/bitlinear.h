@@ -157,8 +157,10 @@ bl_status bitlinear_quant_act(const void* x, bl_dtype xt, int64_t M, int64_t K, 
  *   y        [M][N] row-major, fp32 (yt = BL_F32) or bf16 (BL_BF16), device.
  *   acc_debug  NULL, or int32 [M][N] device buffer that receives acc.
  * fp32 y equals (float)((double)acc * gamma32 / s_m) for M <= 16 (decode
- * kernel); the tensor-core kernel (M > 16) evaluates the same product with
- * a per-token fp64 factor, within 1 fp32 ulp of it.
+ * kernel).  The tensor-core kernel (M > 16) computes fp32(acc) * f_m with
+ * f_m = gamma32 / s_m correctly rounded to fp32: two fp32 roundings, so y
+ * is within 2^-23 relative of that value (bf16 y: equal after rounding
+ * unless the fp32 value sits that close to a bf16 rounding midpoint).
  * Errors: NULL, SHAPE (M, N, K <= 0), ALIGN, DTYPE, OVERFLOW, CUDA.
  * ---------------------------------------------------------------------- */
 bl_status bitlinear_forward(const int8_t* q, const float* s, const uint8_t* packed,
@@ -177,6 +179,27 @@ bl_status bitlinear_forward(const int8_t* q, const float* s, const uint8_t* pack
 bl_status bitlinear_forward_x(const void* x, bl_dtype xt, const uint8_t* packed,
                               const float* gamma32, int64_t M, int64_t N, int64_t K, void* y,
                               bl_dtype yt, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Decode-kernel choice for M <= 16 (bitlinear_forward, bitlinear_forward_x,
+ * bitlinear_forward_x_grouped).  Process-wide, host-side; set it before
+ * launching (and before capturing a CUDA graph).  All kernels give the same
+ * results; the setting exists to compare and test them.
+ *   BL_DECODE_AUTO    M <= 4: dp4a streaming kernel, else tensor-core
+ *                     kernel; M > 4: tensor-core kernel, else dp4a; else the
+ *                     per-tile kernel -- whichever first fits the shapes
+ *   BL_DECODE_TENSOR  tcgen05 kind::i8 kernel with the weights expanded
+ *                     into tensor memory (one CTA per SM)
+ *   BL_DECODE_DP4A    persistent streaming kernel, dp4a on the CUDA cores
+ *   BL_DECODE_TILE    per-tile kernel (the fallback for the largest shapes)
+ * A forced TENSOR or DP4A choice that does not fit the shapes makes the
+ * forward calls return BL_ERR_SHAPE.  bitlinear_set_decode_kernel returns
+ * BL_OK, or BL_ERR_ARG for an unknown value.  The pages define no such
+ * setting: it selects between implementations of the same product.
+ * ---------------------------------------------------------------------- */
+enum { BL_DECODE_AUTO = 0, BL_DECODE_TENSOR = 1, BL_DECODE_DP4A = 2, BL_DECODE_TILE = 3 };
+int bitlinear_set_decode_kernel(int kind);
+int bitlinear_get_decode_kernel(void);
 
 /* ------------------------------------------------------------------------
  * bitlinear_forward_x_grouped -- `count` independent fused BitLinear layers

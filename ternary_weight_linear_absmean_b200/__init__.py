@@ -20,6 +20,7 @@ LIB_PATH = os.path.join(HERE, "libbitlinear.so")
 BL_OK, BL_ERR_NULL, BL_ERR_SHAPE, BL_ERR_ALIGN, BL_ERR_DTYPE = 0, 1, 2, 3, 4
 BL_ERR_WORKSPACE, BL_ERR_OVERFLOW, BL_ERR_NONFINITE, BL_ERR_CUDA, BL_ERR_ARG, BL_ERR_TIMEOUT = 5, 6, 7, 8, 9, 10
 BL_F32, BL_BF16 = 0, 1
+BL_DECODE_AUTO, BL_DECODE_TENSOR, BL_DECODE_DP4A, BL_DECODE_TILE = 0, 1, 2, 3
 
 # Every symbol include/bitlinear.h declares, with (restype, argtypes).
 _vp, _i64, _i32 = C.c_void_p, C.c_int64, C.c_int
@@ -34,6 +35,8 @@ SIGNATURES = {
     "bitlinear_forward_x": (_i32, [_vp, _i32, _vp, _vp, _i64, _i64, _i64, _vp, _i32, _vp]),
     "bitlinear_forward_x_grouped": (_i32, [_i32, _vp, _i32, _vp, _vp, _i64, _vp, _vp, _vp, _i32, _vp]),
     "bitlinear_get_status": (_i32, [_vp]),
+    "bitlinear_set_decode_kernel": (_i32, [_i32]),
+    "bitlinear_get_decode_kernel": (_i32, []),
     "bitlinear_status_string": (C.c_char_p, [_i32]),
 }
 
@@ -174,6 +177,14 @@ def bitlinear_forward_x_grouped(xs, packeds, gammas, Ns, Ks, ys, stream=None) ->
 
 def bitlinear_get_status(stream=None) -> int:
     return int(lib().bitlinear_get_status(_stream(stream)))
+
+
+def bitlinear_set_decode_kernel(kind: int) -> None:
+    _check(lib().bitlinear_set_decode_kernel(int(kind)), "bitlinear_set_decode_kernel")
+
+
+def bitlinear_get_decode_kernel() -> int:
+    return int(lib().bitlinear_get_decode_kernel())
 
 
 bitlinear_status_string = status_string

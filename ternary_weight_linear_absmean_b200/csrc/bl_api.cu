@@ -1,21 +1,51 @@
 // bl_api.cu -- the C ABI of include/bitlinear.h: host-side argument checks,
 // the per-device status word, and dispatch to the kernels.
+#include <atomic>
 #include <cmath>
 #include <cstring>
 
 #include "bl_internal.cuh"
 #include "bl_ptx.cuh"
 
-// One status word per device (the only global state of the library).
+// One status word per device (device-side state of the library).
 __device__ unsigned int g_bl_status_word;
 
 namespace {
+
+// Decode-kernel choice of bitlinear_set_decode_kernel (host-side, process-wide).
+std::atomic<int> g_decode_kernel{BL_DECODE_AUTO};
 
 constexpr int64_t kMaxK = (int64_t(1) << 31) / 127;   // 127*K must stay < 2^31
 constexpr size_t kFusedSmemLimit = 160 * 1024;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool aligned_to(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+// Decode (M <= 16) kernel choice.  AUTO: the dp4a streaming kernel up to 4
+// tokens (measured faster there: its per-byte cost grows with M but starts
+// below the tensor-core kernel's, which is bound by tcgen05 issue), the
+// tensor-core kernel above; each falls back to the next when the shapes do
+// not fit its shared memory.  Returns kTryNext when the per-tile kernel
+// should run.
+constexpr bl_status kTryNext = static_cast<bl_status>(-1);
+
+bl_status dispatch_decode(bl::StreamBatch& sb, bool fused, bl_dtype xt, bl_dtype yt, unsigned* status,
+                          cudaStream_t cs)
+{
+    const int kind = g_decode_kernel.load();
+    if (kind == BL_DECODE_TILE) return kTryNext;
+    const bool tensor_first = kind == BL_DECODE_TENSOR || (kind == BL_DECODE_AUTO && sb.M > 4);
+    for (int pass = 0; pass < 2; ++pass) {
+        const bool tensor = (pass == 0) == tensor_first;
+        if (kind == BL_DECODE_TENSOR && !tensor) break;
+        if (kind == BL_DECODE_DP4A && tensor) continue;
+        bl::StreamBatch b = sb;   // each planner fills its own plan fields
+        const cudaError_t e = tensor ? bl::launch_dec_tc(b, fused, xt, yt, status, cs)
+                                     : bl::launch_stream(b, fused, xt, yt, status, cs);
+        if (e != cudaErrorNotSupported) return e == cudaSuccess ? BL_OK : BL_ERR_CUDA;
+    }
+    return kind == BL_DECODE_AUTO ? kTryNext : BL_ERR_SHAPE;
+}
 
 unsigned* status_word()
 {
@@ -133,8 +163,8 @@ bl_status bitlinear_forward(const int8_t* q, const float* s, const uint8_t* pack
         sb.p[0].acc = acc_debug;
         sb.p[0].N = N;
         sb.p[0].K = K;
-        const cudaError_t e = bl::launch_stream(sb, false, BL_F32, yt, status, cs);
-        if (e != cudaErrorNotSupported) return e == cudaSuccess ? BL_OK : BL_ERR_CUDA;
+        const bl_status r = dispatch_decode(sb, false, BL_F32, yt, status, cs);
+        if (r != kTryNext) return r;
     }
     bl::GemvBatch b;
     std::memset(&b, 0, sizeof(b));
@@ -196,10 +226,19 @@ bl_status bitlinear_forward_x_grouped(int count, const void* const* x, bl_dtype 
         sb.p[i].N = N[i];
         sb.p[i].K = K[i];
     }
-    const cudaError_t e = bl::launch_stream(sb, true, xt, yt, status, cs);
-    if (e != cudaErrorNotSupported) return e == cudaSuccess ? BL_OK : BL_ERR_CUDA;
+    const bl_status r = dispatch_decode(sb, true, xt, yt, status, cs);
+    if (r != kTryNext) return r;
     return bl::launch_gemv(b, true, xt, yt, status, cs) == cudaSuccess ? BL_OK : BL_ERR_CUDA;
 }
+
+int bitlinear_set_decode_kernel(int kind)
+{
+    if (kind < BL_DECODE_AUTO || kind > BL_DECODE_TILE) return BL_ERR_ARG;
+    g_decode_kernel.store(kind);
+    return BL_OK;
+}
+
+int bitlinear_get_decode_kernel(void) { return g_decode_kernel.load(); }
 
 bl_status bitlinear_forward_x(const void* x, bl_dtype xt, const uint8_t* packed, const float* gamma32,
                               int64_t M, int64_t N, int64_t K, void* y, bl_dtype yt, void* stream)

@@ -20,15 +20,17 @@
 //
 // Warp roles (512 threads):
 //   warp 0       TMEM allocation; TMA producer (one lane)
-//   warp 1       MMA issuer (one lane): 8 x tcgen05.mma (K = 32) per stage,
+//   warps 1, 2   MMA issuers (one lane each, tokens 0-63 and 64-127 of the
+//                tile): 8 x tcgen05.mma (N = 64, K = 32) per stage,
 //                tcgen05.commit -> stage-free barrier; per tile -> acc-full.
-//                It waits only for the expansion barrier: the expansion
+//                They wait only for the expansion barrier: the expansion
 //                threads arrive there after observing the stage's TMA
 //                barrier, so the activation tile is complete by then too
 //   warps 4-11   expansion, two groups of four taking alternate stages:
 //                warp w writes TMEM lanes 32*(w%4) .. +31 of its stages
-//   warps 12-15  epilogue: per-token factors gamma32 / s_m (fp64),
-//                tcgen05.ld of the finished accumulator, rescale, store y,
+//   warps 12-15  epilogue: per-token factors f_m = gamma32 / s_m (fp32,
+//                correctly rounded), tcgen05.ld of the finished accumulator,
+//                y = fp32(acc) * f_m (the conversion is exact below 2^24), store,
 //                then release the accumulator
 // All mbarrier waits are bounded (bl_ptx.cuh); every role reaches the final
 // barrier, after which the allocating warp frees the tensor memory.
@@ -41,6 +43,7 @@
 
 #include "bl_internal.cuh"
 #include "bl_ptx.cuh"
+#include "bl_tc.cuh"
 
 namespace bl {
 namespace {
@@ -63,7 +66,6 @@ constexpr int EXP_WARP0 = 4, EPI_WARP0 = 12;
 struct Smem {
     uint8_t q[STAGES][Q_STAGE];              // 1024-aligned (first member)
     uint8_t w[STAGES][W_STAGE];
-    double fac[2][BN];
     uint64_t full[STAGES], expanded[STAGES], empty[STAGES];
     uint64_t acc_full[2], acc_empty[2], done;
     uint32_t tmem_base;
@@ -79,74 +81,29 @@ __device__ __forceinline__ uint32_t signed_codes(int t, uint32_t w)
     return (((w >> (2 * t)) & 0x03030303u) + 0x7F7F7F7Fu) ^ 0x80808080u;
 }
 
-__device__ __forceinline__ uint64_t make_bdesc(uint32_t smem_addr)
-{
-    // K-major, 128-byte swizzle: rows of 128 B, 8-row core groups 1024 B apart.
-    uint64_t d = 0;
-    d |= (uint64_t)((smem_addr >> 4) & 0x3FFF);          // start address
-    d |= (uint64_t)1 << 16;                               // leading byte offset (unused for SW128 K-major)
-    d |= (uint64_t)(1024 >> 4) << 32;                     // stride byte offset
-    d |= (uint64_t)1 << 46;                               // descriptor version (sm_100)
-    d |= (uint64_t)2 << 61;                               // SWIZZLE_128B
-    return d;
-}
-
-// kind::i8, D = S32, A = B = signed int8, both K-major, M = 128, N = BN.
-constexpr uint32_t kIdesc = (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
-                            ((uint32_t)(BM >> 4) << 24);
-
-__device__ __forceinline__ void mma_i8_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t accumulate)
-{
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_tmem), "l"(b_desc), "r"(kIdesc), "r"(accumulate)
-        : "memory");
-}
-
-__device__ __forceinline__ void mma_commit(uint64_t* bar)
-{
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                     smem_u32(bar))
-                 : "memory");
-}
-
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32])
-{
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, "
-        "%13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(
-            taddr),
-        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
-        "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]),
-        "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]),
-        "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
-        : "memory");
-}
-
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32])
-{
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
-        "%14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
-        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
-          "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]),
-          "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]),
-          "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]),
-          "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
-        : "r"(taddr)
-        : "memory");
-}
-
-__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
-__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+// kind::i8, D = S32, A = B = signed int8, both K-major, M = 128, N = BN/2:
+// two issuing threads each take half of the tokens (one thread issues a
+// tcgen05.mma only every ~57 cycles; two keep the tensor pipe busy).
+constexpr int HALF_N = BN / 2;
+constexpr uint32_t kIdesc = idesc_i8(BM, HALF_N);
 
 __device__ __forceinline__ void store_y(float* y, int64_t i, float v) { y[i] = v; }
-__device__ __forceinline__ void store_y(__nv_bfloat16* y, int64_t i, float v) { y[i] = __float2bfloat16_rn(v); }
+// bf16 round-to-nearest-even on the bit pattern (y is always finite here):
+// add 0x7FFF plus the lowest kept bit, then truncate.
+__device__ __forceinline__ void store_y(__nv_bfloat16* y, int64_t i, float v)
+{
+    uint32_t u = __float_as_uint(v);
+    u += 0x7FFFu + ((u >> 16) & 1u);
+    reinterpret_cast<uint16_t*>(y)[i] = (uint16_t)(u >> 16);
+}
+
+// int32 -> fp32, exact for |a| < 2^22 with two ALU-pipe instructions: the
+// float with bit pattern 0x4B400000 + a is 1.5 * 2^23 + a (its unit in the
+// last place is 1), and subtracting 1.5 * 2^23 leaves a.
+__device__ __forceinline__ float small_int_to_float(int a)
+{
+    return __fsub_rn(__int_as_float(0x4B400000 + a), 12582912.0f);
+}
 
 template <typename YT>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -155,6 +112,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
                YT* __restrict__ y, int32_t* __restrict__ acc_out, unsigned* status)
 {
     extern __shared__ uint8_t smem_raw[];
+    // per-token factors gamma32 / s_m of the two accumulator buffers; a
+    // static array, so the compiler sees shared-memory loads it may batch
+    __shared__ float s_fac[2][BN];
     Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int tiles_n = (N + BM - 1) / BM, tiles_m = (M + BN - 1) / BN;
@@ -164,13 +124,13 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&sm.full[s], 1);
             mbar_init(&sm.expanded[s], 128);   // one expansion group
-            mbar_init(&sm.empty[s], 1);
+            mbar_init(&sm.empty[s], 2);
         }
         for (int b = 0; b < 2; ++b) {
-            mbar_init(&sm.acc_full[b], 1);
+            mbar_init(&sm.acc_full[b], 2);
             mbar_init(&sm.acc_empty[b], 128);
         }
-        mbar_init(&sm.done, 1);
+        mbar_init(&sm.done, 2);
         sm.abort_flag = 0;
         fence_barrier_init();
     }
@@ -214,16 +174,19 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
             for (int j = g - STAGES < 0 ? 0 : g - STAGES; j < g; ++j)
                 wait_parity(&sm.full[j % STAGES], (j / STAGES) & 1, status, nullptr, true);
         }
-    } else if (warp == 1) {
-        // ------------------------------------------------------ MMA issuer
+    } else if (warp == 1 || warp == 2) {
+        // ----------------------------------------------------- MMA issuers
+        // warp 1: tokens 0..63 of the tile, warp 2: tokens 64..127 (B rows
+        // 64.. start 8 swizzle groups = 8 KiB into each slab; D columns 64..)
         if (lane == 0) {
+            const int hn = warp - 1;
             int g = 0, i = 0;
             bool ok = true;
             for (int t = blockIdx.x; ok && t < total; t += gridDim.x, ++i) {
                 const int b = i & 1, ar = i >> 1;
                 if (ar > 0 && !wait_parity(&sm.acc_empty[b], (ar - 1) & 1, status, abort)) break;
                 tc_fence_after();
-                const uint32_t d_tmem = tmem + b * ACC_COLS;
+                const uint32_t d_tmem = tmem + b * ACC_COLS + hn * HALF_N;
                 for (int kb = 0; kb < nk; ++kb, ++g) {
                     const int s = g % STAGES;
                     const uint32_t ph = (g / STAGES) & 1;
@@ -232,11 +195,11 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t qaddr = smem_u32(sm.q[s]);
+                    const uint32_t qaddr = smem_u32(sm.q[s]) + hn * (HALF_N / 8) * 1024;
 #pragma unroll
                     for (int j = 0; j < BK / 32; ++j)
                         mma_i8_ts(d_tmem, tmem + A_COL0 + s * A_STAGE_COLS + j * 8,
-                                  make_bdesc(qaddr + (j >> 2) * Q_ATOM + (j & 3) * 32), (kb | j) != 0);
+                                  make_bdesc(qaddr + (j >> 2) * Q_ATOM + (j & 3) * 32), kIdesc, (kb | j) != 0);
                     mma_commit(&sm.empty[s]);
                 }
                 if (ok) mma_commit(&sm.acc_full[b]);
@@ -290,14 +253,16 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
         const int quarter = warp & 3;
         const int rr = 32 * quarter + lane;
         const uint32_t lane_base = (uint32_t)(32 * quarter) << 16;
-        const double gam = (double)*gamma32;
+        const float gam = *gamma32;
+        // |acc| <= 127 * Kp: below 2^22 the conversion needs no converter unit
+        const bool small_acc = (int64_t)127 * nk * BK < (int64_t(1) << 22);
         int i = 0;
         for (int t = blockIdx.x; t < total; t += gridDim.x, ++i) {
             const int b = i & 1, ar = i >> 1;
             const int n0 = (t % tiles_n) * BM, m0 = (t / tiles_n) * BN;
             {
                 const int m = m0 + et;
-                sm.fac[b][et] = (m < M) ? gam / (double)s_in[m] : 0.0;
+                s_fac[b][et] = (m < M) ? __fdiv_rn(gam, s_in[m]) : 0.0f;
             }
             // one thread waits for the accumulator; the verdict goes through
             // shared memory so all four warps take the same branch
@@ -313,15 +278,29 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
                 tmem_ld32(acc_tmem + cc * 32, v);
                 tmem_wait_ld();
                 if (n < N) {
+                    // 8 tokens at a time: factors first (independent
+                    // loads), then 8 independent rescale chains, then the
+                    // stores, so no load waits behind a store
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        const int m = m0 + cc * 32 + j;
-                        if (m < M) {
-                            const int a = (int)v[j];
-                            const int64_t o = (int64_t)m * N + n;
-                            if (acc_out) acc_out[o] = a;
-                            store_y(y, o, (float)((double)a * sm.fac[b][cc * 32 + j]));
+                    for (int h = 0; h < 4; ++h) {
+                        float f[8];
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) f[j] = s_fac[b][cc * 32 + h * 8 + j];
+                        float o[8];
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            const int a = (int)v[h * 8 + j];
+                            o[j] = __fmul_rn(small_acc ? small_int_to_float(a) : __int2float_rn(a), f[j]);
                         }
+                        const int mb = m0 + cc * 32 + h * 8;
+                        if (acc_out) {
+#pragma unroll
+                            for (int j = 0; j < 8; ++j)
+                                if (mb + j < M) acc_out[(int64_t)(mb + j) * N + n] = (int)v[h * 8 + j];
+                        }
+#pragma unroll
+                        for (int j = 0; j < 8; ++j)
+                            if (mb + j < M) store_y(y, (int64_t)(mb + j) * N + n, o[j]);
                     }
                 }
             }

@@ -90,6 +90,7 @@ struct StreamBatch {
     int M;
     int stages;             // set by plan_stream
     int q_bytes;            // set by plan_stream
+    int layout_tokens;      // tensor-core kernel: token slots of its operand layout
 };
 constexpr int kMaxStages = 12;
 // dynamic shared memory per CTA for `minb` resident CTAs per SM
@@ -99,6 +100,13 @@ int sm_count();
 bool plan_stream(StreamBatch& b, int minb, int* grid, size_t* smem);
 // Returns cudaErrorNotSupported if the shapes do not fit (shared memory).
 cudaError_t launch_stream(StreamBatch& b, bool fused, bl_dtype xt, bl_dtype yt, unsigned* status,
+                          cudaStream_t st);
+
+// Tensor-core decode kernel (bl_decode_tc.cu), M <= 16: same batch as the
+// streaming kernel (plan fields are filled by its own planner).  Returns
+// cudaErrorNotSupported if the shapes do not fit (shared memory).
+bool plan_dec_tc(StreamBatch& b, int* grid, size_t* smem);
+cudaError_t launch_dec_tc(StreamBatch& b, bool fused, bl_dtype xt, bl_dtype yt, unsigned* status,
                           cudaStream_t st);
 
 // Prefill tensor-core GEMM (tcgen05 kind::i8).  Returns cudaErrorNotSupported

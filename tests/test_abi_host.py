@@ -99,3 +99,13 @@ def test_forward_x_rejects_bad_arguments(L):
     assert g(17, arr, bl.BL_BF16, arr, arr, 1, i64, i64, arr, bl.BL_F32, None) == bl.BL_ERR_ARG
     bad = (C.c_void_p * 2)(A, None)
     assert g(2, bad, bl.BL_BF16, arr, arr, 1, i64, i64, arr, bl.BL_F32, None) == bl.BL_ERR_NULL
+
+
+def test_decode_kernel_setting_is_host_only(L):
+    # process-wide choice; no CUDA call behind it
+    assert L.bitlinear_get_decode_kernel() == bl.BL_DECODE_AUTO
+    for k in (bl.BL_DECODE_TENSOR, bl.BL_DECODE_DP4A, bl.BL_DECODE_TILE, bl.BL_DECODE_AUTO):
+        assert L.bitlinear_set_decode_kernel(k) == bl.BL_OK
+        assert L.bitlinear_get_decode_kernel() == k
+    assert L.bitlinear_set_decode_kernel(7) == bl.BL_ERR_ARG
+    assert L.bitlinear_get_decode_kernel() == bl.BL_DECODE_AUTO
