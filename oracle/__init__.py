@@ -69,6 +69,10 @@ def lib() -> C.CDLL:
             L.orc_quant_act_f32.argtypes = [vp, i64, i64, vp, vp]
             L.orc_quant_act_bf16.restype = i64
             L.orc_quant_act_bf16.argtypes = [vp, i64, i64, vp, vp]
+            L.orc_rms_factor.restype = C.c_float
+            L.orc_rms_factor.argtypes = [vp, i64, C.c_double]
+            L.orc_rmsnorm_quant_act.restype = i64
+            L.orc_rmsnorm_quant_act.argtypes = [vp, C.c_int, vp, C.c_double, i64, i64, vp, vp, vp]
             L.orc_int_matmul.restype = C.c_int
             L.orc_int_matmul.argtypes = [vp, vp, i64, i64, i64, vp]
             L.orc_int_matmul_sampled.restype = C.c_int
@@ -170,6 +174,36 @@ def quant_act(x: np.ndarray, dtype: str):
     return q, s, int(clipped)
 
 
+def rms_factor(x_row: np.ndarray, eps: float) -> np.float32:
+    """r32 = (float)(1 / sqrt(mean(x^2) + eps)), mean square summed in fp64."""
+    x_row = _c(x_row, np.float32)
+    return np.float32(lib().orc_rms_factor(_p(x_row), x_row.size, float(eps)))
+
+
+def rmsnorm_quant_act(x: np.ndarray, dtype: str, gain: np.ndarray, eps: float):
+    """SubLN (RMS normalisation with per-channel gain) then the per-token
+    int8 quantiser.  x as in quant_act.  Returns (xn float32 [M, K], q int8
+    [M, K], s float32 [M], clipped count)."""
+    if dtype == "f32":
+        x = _c(x, np.float32)
+        xt = 0
+    elif dtype == "bf16":
+        x = _c(x, np.uint16)
+        xt = 1
+    else:
+        raise ValueError(dtype)
+    M, K = x.shape
+    gain = _c(gain, np.float32)
+    assert gain.shape == (K,)
+    xn = np.empty((M, K), np.float32)
+    q = np.empty((M, K), np.int8)
+    s = np.empty(M, np.float32)
+    clipped = lib().orc_rmsnorm_quant_act(_p(x), xt, _p(gain), float(eps), M, K, _p(xn), _p(q), _p(s))
+    if clipped < 0:
+        raise MemoryError("oracle rmsnorm_quant_act allocation failed")
+    return xn, q, s, int(clipped)
+
+
 # ---------------------------------------------------------------- A4 ----
 def int_matmul(q: np.ndarray, code: np.ndarray) -> np.ndarray:
     q = _c(q, np.int8)
@@ -228,6 +262,19 @@ def bitlinear(W: np.ndarray, x: np.ndarray, xdtype: str, eps: float = 1e-5):
     y = rescale(acc, s, g32)
     return dict(gamma64=g64, gamma32=g32, code=code, boundary=bnd, n_boundary=nb,
                 packed=pack(code), q=q, s=s, clipped=clipped, acc=acc, y=y)
+
+
+def bitlinear_rmsnorm(W: np.ndarray, x: np.ndarray, xdtype: str, gain: np.ndarray, eps_norm: float,
+                      eps: float = 1e-5):
+    """SubLN (RMS normalisation, reading R16) then the whole layer."""
+    g64 = absmean_gamma(W)
+    g32 = float(np.float32(g64))
+    code, bnd, nb = ternary_codes(W, g64, eps)
+    xn, q, s, clipped = rmsnorm_quant_act(x, xdtype, gain, eps_norm)
+    acc = int_matmul(q, code)
+    y = rescale(acc, s, g32)
+    return dict(gamma64=g64, gamma32=g32, code=code, boundary=bnd, n_boundary=nb,
+                packed=pack(code), xn=xn, q=q, s=s, clipped=clipped, acc=acc, y=y)
 
 
 def forward_bf16_mt(x_bf16: np.ndarray, code: np.ndarray, gamma32: float, threads: int) -> np.ndarray:

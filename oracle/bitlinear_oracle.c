@@ -27,6 +27,9 @@
  *       would have.
  *   R6  s = 127 / amax is a multiplier, so the rescale divides by s.
  *   R10 y is fp32: (float)((double)acc * (double)gamma32 / (double)s).
+ *   R16 SubLN = RMS normalisation with a per-channel gain; the mean square
+ *       is summed in fp64 and the factor rounded once to fp32 (see
+ *       orc_rms_factor).
  *
  * Build: gcc -O2 -std=c11 -ffp-contract=off -fno-fast-math -fPIC -shared
  * (no FMA contraction: every float operation below rounds exactly once, in
@@ -202,6 +205,55 @@ int64_t orc_quant_act_bf16(const uint16_t* x, int64_t M, int64_t K, int8_t* q, f
     for (int64_t m = 0; m < M; ++m) {
         for (int64_t k = 0; k < K; ++k) row[k] = orc_bf16_to_f32(x[m * K + k]);
         clipped += orc_quant_row(row, K, q + m * K, s + m);
+    }
+    free(row);
+    return clipped;
+}
+
+/* ------------------------------------------------------------------------ */
+/* SubLN before the activation quantiser.                                   */
+/* [ARATECH] "BitLinear: the building block": a sub-layer normalisation, a  */
+/* simplified variant of LayerNorm, sits before the activation quantisation */
+/* for training stability; the page does not define it further.  Reading   */
+/* R16: the simplified LayerNorm is RMS normalisation (no mean subtraction, */
+/* no bias) with a per-channel gain g:                                      */
+/*   ms   = (sum_k x_k^2) / K           fp64 (each square is exact in fp64, */
+/*                                      summed left to right)               */
+/*   r    = 1 / sqrt(ms + eps)          fp64, then rounded to fp32 (r32)    */
+/*   xn_k = (x_k * r32) * g_k           fp32, two roundings, in that order  */
+/* and xn is then quantised exactly like x (orc_quant_row).                 */
+/* ------------------------------------------------------------------------ */
+float orc_rms_factor(const float* x, int64_t K, double eps)
+{
+    double ss = 0.0;
+    for (int64_t k = 0; k < K; ++k) ss += (double)x[k] * (double)x[k];
+    const double r = 1.0 / sqrt(ss / (double)K + eps);
+    return (float)r;
+}
+
+void orc_rmsnorm_row(const float* x, int64_t K, const float* g, double eps, float* xn)
+{
+    const float r32 = orc_rms_factor(x, K, eps);
+    for (int64_t k = 0; k < K; ++k) {
+        const float t = x[k] * r32;   /* rounds once (no contraction) */
+        xn[k] = t * g[k];             /* rounds once */
+    }
+}
+
+/* x given as fp32 (xt = 0) or bf16 bit patterns (xt = 1); writes the fp32   */
+/* normalised rows, then q and s as orc_quant_act_*.  Returns the clipped    */
+/* count, or -1 on allocation failure.                                       */
+int64_t orc_rmsnorm_quant_act(const void* x, int xt, const float* g, double eps, int64_t M, int64_t K,
+                              float* xn, int8_t* q, float* s)
+{
+    float* row = (float*)malloc((size_t)K * sizeof(float));
+    if (!row) return -1;
+    int64_t clipped = 0;
+    for (int64_t m = 0; m < M; ++m) {
+        for (int64_t k = 0; k < K; ++k)
+            row[k] = xt ? orc_bf16_to_f32(((const uint16_t*)x)[m * K + k]) : ((const float*)x)[m * K + k];
+        orc_rmsnorm_row(row, K, g, eps, xn + m * K);
+        clipped += orc_quant_row(xn + m * K, K, q + m * K, s + m);
     }
     free(row);
     return clipped;

@@ -336,3 +336,88 @@ def test_synth_weights_recipe_and_distribution():
     assert np.array_equal(big[:3], oracle.synth_weights(1, 0, 0, 3, 1024))
     assert abs(float(big.mean())) < 1e-4
     assert abs(float(big.std()) - 0.02) < 2e-4
+
+
+# ------------------------------------------------------------ SubLN (R16)
+# RMS normalisation before the quantiser, pinned against torch's own
+# rms_norm (a library routine, run in fp64), closed forms and invariants.
+
+def _torch_rms_norm_f64(x, g, eps):
+    import torch
+    t = torch.from_numpy(np.asarray(x, np.float64))
+    return torch.nn.functional.rms_norm(t, (t.shape[-1],), torch.from_numpy(np.asarray(g, np.float64)),
+                                        eps).numpy()
+
+
+@pytest.mark.parametrize("K,eps", [(1, 1e-6), (7, 1e-6), (512, 1e-6), (2560, 1e-5), (64, 1e-2)])
+def test_rmsnorm_matches_library_rms_norm(K, eps):
+    rng = np.random.default_rng(K)
+    x = (rng.standard_normal((3, K)) * np.array([[1.0], [0.05], [3.0]])).astype(np.float32)
+    g = (1.0 + 0.1 * rng.standard_normal(K)).astype(np.float32)
+    xn, q, s, clipped = oracle.rmsnorm_quant_act(x, "f32", g, eps)
+    ref = _torch_rms_norm_f64(x, g, eps)
+    # three fp32 roundings (the factor, x*r, *g): within 2^-22 relative
+    assert np.all(np.abs(xn - ref) <= 2.0 ** -22 * np.abs(ref) + 1e-30)
+    # the quantiser then runs on xn exactly as on any input
+    q2, s2, _ = oracle.quant_act(xn, "f32")
+    assert np.array_equal(q, q2) and np.array_equal(s, s2) and clipped == 0
+
+
+def test_rmsnorm_eps_inside_the_root():
+    # small-magnitude row where eps dominates: sqrt(ms + eps), not sqrt(ms) + eps
+    x = np.full((1, 16), 1e-3, np.float32)
+    g = np.ones(16, np.float32)
+    xn, _, _, _ = oracle.rmsnorm_quant_act(x, "f32", g, 1e-2)
+    want = 1e-3 / np.sqrt(1e-6 + 1e-2)
+    assert abs(float(xn[0, 0]) - want) <= 2.0 ** -22 * want
+
+
+def test_rmsnorm_constant_row_and_unit_rms():
+    g = np.ones(300, np.float32)
+    for c in (0.75, -3.0, 1e-4, 123.0):
+        x = np.full((1, 300), c, np.float32)
+        xn, _, _, _ = oracle.rmsnorm_quant_act(x, "f32", g, 0.0)
+        assert np.all(np.abs(np.abs(xn) - 1.0) <= 2.0 ** -22)
+        assert np.all(np.sign(xn) == np.sign(c))
+    rng = np.random.default_rng(3)
+    x = rng.standard_normal((4, 1000)).astype(np.float32)
+    xn, _, _, _ = oracle.rmsnorm_quant_act(x, "f32", np.ones(1000, np.float32), 0.0)
+    ms = (xn.astype(np.float64) ** 2).mean(axis=1)
+    assert np.all(np.abs(ms - 1.0) < 1e-6)
+
+
+def test_rmsnorm_power_of_two_scaling_is_exact():
+    # eps = 0: scaling x by 2^j scales the mean square by 4^j exactly, so the
+    # factor by 2^-j and every normalised value is bit-identical; a gain of
+    # 2^i scales the output exactly
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal((2, 777)).astype(np.float32)
+    g = (1 + 0.2 * rng.standard_normal(777)).astype(np.float32)
+    a, qa, sa, _ = oracle.rmsnorm_quant_act(x, "f32", g, 0.0)
+    b, qb, sb, _ = oracle.rmsnorm_quant_act(x * np.float32(8.0), "f32", g, 0.0)
+    assert np.array_equal(a.view(np.uint32), b.view(np.uint32))
+    assert np.array_equal(qa, qb) and np.array_equal(sa, sb)
+    c, _, _, _ = oracle.rmsnorm_quant_act(x, "f32", g * np.float32(0.25), 0.0)
+    assert np.array_equal((a * np.float32(0.25)).view(np.uint32), c.view(np.uint32))
+
+
+def test_rmsnorm_permutation_equivariant_on_exact_sums():
+    # small integers: every fp64 partial sum is exact, so the order of the
+    # sum cannot matter and a permuted row gives the permuted result
+    rng = np.random.default_rng(9)
+    x = rng.integers(-20, 21, size=(1, 256)).astype(np.float32)
+    g = (1 + 0.3 * rng.standard_normal(256)).astype(np.float32)
+    perm = rng.permutation(256)
+    a, _, _, _ = oracle.rmsnorm_quant_act(x, "f32", g, 1e-6)
+    b, _, _, _ = oracle.rmsnorm_quant_act(x[:, perm], "f32", g[perm], 1e-6)
+    assert np.array_equal(a[:, perm].view(np.uint32), b.view(np.uint32))
+
+
+def test_rmsnorm_bf16_input_is_widened_exactly():
+    rng = np.random.default_rng(11)
+    xf = rng.standard_normal((2, 300)).astype(np.float32)
+    bits = synth.f32_to_bf16_bits(xf)
+    g = np.ones(300, np.float32)
+    a, qa, sa, _ = oracle.rmsnorm_quant_act(bits, "bf16", g, 1e-6)
+    b, qb, sb, _ = oracle.rmsnorm_quant_act(synth.bf16_bits_to_f32(bits), "f32", g, 1e-6)
+    assert np.array_equal(a, b) and np.array_equal(qa, qb) and np.array_equal(sa, sb)
