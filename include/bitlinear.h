@@ -181,6 +181,36 @@ bl_status bitlinear_forward_x(const void* x, bl_dtype xt, const uint8_t* packed,
                               bl_dtype yt, void* stream);
 
 /* ------------------------------------------------------------------------
+ * SubLN before the activation quantiser.  aratech.ae, "BitLinear: the
+ * building block": a sub-layer normalisation, a simplified LayerNorm, sits
+ * before the activation quantisation.  The page does not define it further;
+ * it is read here as RMS normalisation with a per-channel gain g [K]:
+ *   r = fp32(1 / sqrt(sum_k x_k^2 / K + eps))   (the sum in fp64)
+ *   x_k <- (x_k * r) * g_k                       (fp32, rounded in that order)
+ * followed by the per-token absmax quantiser of bitlinear_quant_act.  The
+ * sum's order differs from a sequential sum by ~1e-16 relative, so r (and
+ * then q, s) can differ from another implementation's only when r lies that
+ * close to an fp32 rounding midpoint.
+ *
+ * bitlinear_rmsnorm_quant_act -- the normalisation and the quantiser in one
+ *   kernel: arguments as bitlinear_quant_act plus gain (fp32 [K], device,
+ *   16-byte aligned) and eps (>= 0, finite, else BL_ERR_ARG).
+ * bitlinear_forward_x_rmsnorm_grouped -- the fused decode form of
+ *   bitlinear_forward_x_grouped with the normalisation in the prologue; each
+ *   problem i has its own x[i] and gain[i] (pass the same pointers for
+ *   linears that share one normalised input).  Same limits as that call
+ *   (M <= 16, M' * Kp <= 160 KiB); BL_ERR_SHAPE also when neither streaming
+ *   decode kernel fits, or when the per-tile kernel is forced (it has no
+ *   normalising prologue).
+ * ---------------------------------------------------------------------- */
+bl_status bitlinear_rmsnorm_quant_act(const void* x, bl_dtype xt, const float* gain, double eps, int64_t M,
+                                      int64_t K, int8_t* q, float* s, void* stream);
+bl_status bitlinear_forward_x_rmsnorm_grouped(int count, const void* const* x, bl_dtype xt,
+                                              const float* const* gain, double eps, const uint8_t* const* packed,
+                                              const float* const* gamma32, int64_t M, const int64_t* N,
+                                              const int64_t* K, void* const* y, bl_dtype yt, void* stream);
+
+/* ------------------------------------------------------------------------
  * Decode-kernel choice for M <= 16 (bitlinear_forward, bitlinear_forward_x,
  * bitlinear_forward_x_grouped).  Process-wide, host-side; set it before
  * launching (and before capturing a CUDA graph).  All kernels give the same

@@ -34,6 +34,9 @@ SIGNATURES = {
     "bitlinear_forward": (_i32, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _i32, _vp, _vp]),
     "bitlinear_forward_x": (_i32, [_vp, _i32, _vp, _vp, _i64, _i64, _i64, _vp, _i32, _vp]),
     "bitlinear_forward_x_grouped": (_i32, [_i32, _vp, _i32, _vp, _vp, _i64, _vp, _vp, _vp, _i32, _vp]),
+    "bitlinear_rmsnorm_quant_act": (_i32, [_vp, _i32, _vp, C.c_double, _i64, _i64, _vp, _vp, _vp]),
+    "bitlinear_forward_x_rmsnorm_grouped": (_i32, [_i32, _vp, _i32, _vp, C.c_double, _vp, _vp, _i64, _vp, _vp,
+                                                   _vp, _i32, _vp]),
     "bitlinear_get_status": (_i32, [_vp]),
     "bitlinear_set_decode_kernel": (_i32, [_i32]),
     "bitlinear_get_decode_kernel": (_i32, []),
@@ -175,6 +178,27 @@ def bitlinear_forward_x_grouped(xs, packeds, gammas, Ns, Ks, ys, stream=None) ->
     _check(st, "bitlinear_forward_x_grouped")
 
 
+def bitlinear_rmsnorm_quant_act(x, gain, eps, q, s, stream=None) -> None:
+    M, K = x.shape
+    st = lib().bitlinear_rmsnorm_quant_act(_dptr(x, "x"), _dtype_code(x.dtype), _dptr(gain, "gain"), float(eps), M,
+                                           K, _dptr(q, "q"), _dptr(s, "s"), _stream(stream))
+    _check(st, "bitlinear_rmsnorm_quant_act")
+
+
+def bitlinear_forward_x_rmsnorm_grouped(xs, gains, eps, packeds, gammas, Ns, Ks, ys, stream=None) -> None:
+    n = len(xs)
+    if not (len(gains) == len(packeds) == len(gammas) == len(Ns) == len(Ks) == len(ys) == n):
+        raise ValueError("grouped arguments must all have the same length")
+    M = xs[0].shape[0]
+    arr_p = C.c_void_p * n
+    arr_i = C.c_int64 * n
+    st = lib().bitlinear_forward_x_rmsnorm_grouped(
+        n, arr_p(*[_dptr(t, "x") for t in xs]), _dtype_code(xs[0].dtype), arr_p(*[_dptr(t, "gain") for t in gains]),
+        float(eps), arr_p(*[_dptr(t, "packed") for t in packeds]), arr_p(*[_dptr(t, "gamma32") for t in gammas]),
+        M, arr_i(*Ns), arr_i(*Ks), arr_p(*[_dptr(t, "y") for t in ys]), _dtype_code(ys[0].dtype), _stream(stream))
+    _check(st, "bitlinear_forward_x_rmsnorm_grouped")
+
+
 def bitlinear_get_status(stream=None) -> int:
     return int(lib().bitlinear_get_status(_stream(stream)))
 
@@ -211,6 +235,17 @@ def quant_act(x, stream=None):
     q = torch.empty((M, bitlinear_padded_k(K)), dtype=torch.int8, device=x.device)
     s = torch.empty(M, dtype=torch.float32, device=x.device)
     bitlinear_quant_act(x, q, s, stream)
+    return q, s
+
+
+def rmsnorm_quant_act(x, gain, eps: float = 1e-6, stream=None):
+    """SubLN (RMS normalisation with gain) then the quantiser.  Returns
+    (q int8 [M, Kp], s float32 [M])."""
+    torch = _torch()
+    M, K = x.shape
+    q = torch.empty((M, bitlinear_padded_k(K)), dtype=torch.int8, device=x.device)
+    s = torch.empty(M, dtype=torch.float32, device=x.device)
+    bitlinear_rmsnorm_quant_act(x, gain, eps, q, s, stream)
     return q, s
 
 

@@ -132,6 +132,23 @@ bl_status bitlinear_quant_act(const void* x, bl_dtype xt, int64_t M, int64_t K, 
                : BL_ERR_CUDA;
 }
 
+bl_status bitlinear_rmsnorm_quant_act(const void* x, bl_dtype xt, const float* gain, double eps, int64_t M,
+                                      int64_t K, int8_t* q, float* s, void* stream)
+{
+    if (!x || !gain || !q || !s) return BL_ERR_NULL;
+    if (check_dtype(xt) != BL_OK) return BL_ERR_DTYPE;
+    if (M <= 0 || K <= 0 || M > (int64_t(1) << 31) - 1) return BL_ERR_SHAPE;
+    if (K > kMaxK) return BL_ERR_OVERFLOW;
+    if (!aligned16(x) || !aligned16(q) || !aligned16(s) || !aligned16(gain)) return BL_ERR_ALIGN;
+    if (!(eps >= 0.0) || !std::isfinite(eps)) return BL_ERR_ARG;
+    unsigned* status = status_word();
+    if (!status) return BL_ERR_CUDA;
+    return bl::launch_rmsnorm_quant(x, xt, gain, eps, M, K, q, s, status, static_cast<cudaStream_t>(stream)) ==
+                   cudaSuccess
+               ? BL_OK
+               : BL_ERR_CUDA;
+}
+
 bl_status bitlinear_forward(const int8_t* q, const float* s, const uint8_t* packed,
                             const float* gamma32, int64_t M, int64_t N, int64_t K, void* y,
                             bl_dtype yt, int32_t* acc_debug, void* stream)
@@ -239,6 +256,47 @@ int bitlinear_set_decode_kernel(int kind)
 }
 
 int bitlinear_get_decode_kernel(void) { return g_decode_kernel.load(); }
+
+bl_status bitlinear_forward_x_rmsnorm_grouped(int count, const void* const* x, bl_dtype xt,
+                                              const float* const* gain, double eps, const uint8_t* const* packed,
+                                              const float* const* gamma32, int64_t M, const int64_t* N,
+                                              const int64_t* K, void* const* y, bl_dtype yt, void* stream)
+{
+    if (count < 1 || count > bl::kMaxGroup) return BL_ERR_ARG;
+    if (!x || !gain || !packed || !gamma32 || !N || !K || !y) return BL_ERR_NULL;
+    if (check_dtype(xt) != BL_OK || check_dtype(yt) != BL_OK) return BL_ERR_DTYPE;
+    if (M <= 0 || M > bl::kFusedMaxM) return BL_ERR_SHAPE;
+    if (!(eps >= 0.0) || !std::isfinite(eps)) return BL_ERR_ARG;
+    bl::StreamBatch sb;
+    std::memset(&sb, 0, sizeof(sb));
+    sb.count = count;
+    sb.M = (int)M;
+    sb.eps_norm = eps;
+    int64_t tiles = 0;
+    for (int i = 0; i < count; ++i) {
+        if (!x[i] || !gain[i] || !packed[i] || !gamma32[i] || !y[i]) return BL_ERR_NULL;
+        bl_status st = check_forward_shape(M, N[i], K[i]);
+        if (st != BL_OK) return st;
+        if ((size_t)pow2_tokens(M) * (size_t)bl::padded_k(K[i]) > kFusedSmemLimit) return BL_ERR_SHAPE;
+        if (!aligned16(x[i]) || !aligned16(gain[i]) || !aligned16(packed[i]) || !aligned_to(gamma32[i], 4) ||
+            !aligned16(y[i]))
+            return BL_ERR_ALIGN;
+        tiles += bl::padded_n(N[i]) / 8;
+        sb.p[i].x = x[i];
+        sb.p[i].gain = gain[i];
+        sb.p[i].packed = packed[i];
+        sb.p[i].gamma32 = gamma32[i];
+        sb.p[i].y = y[i];
+        sb.p[i].N = N[i];
+        sb.p[i].K = K[i];
+    }
+    if (tiles > (int64_t(1) << 31) - 1) return BL_ERR_SHAPE;
+    unsigned* status = status_word();
+    if (!status) return BL_ERR_CUDA;
+    const bl_status r = dispatch_decode(sb, true, xt, yt, status, static_cast<cudaStream_t>(stream));
+    // the per-tile kernel has no normalising prologue
+    return r == kTryNext ? BL_ERR_SHAPE : r;
+}
 
 bl_status bitlinear_forward_x(const void* x, bl_dtype xt, const uint8_t* packed, const float* gamma32,
                               int64_t M, int64_t N, int64_t K, void* y, bl_dtype yt, void* stream)

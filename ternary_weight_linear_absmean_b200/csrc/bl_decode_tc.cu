@@ -143,6 +143,19 @@ __device__ __forceinline__ uint32_t pro_max(uint32_t v, int* red)
     return m;
 }
 
+__device__ __forceinline__ double pro_sum_f64(double v, double* red)
+{
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    const int w = (threadIdx.x >> 5) - kExpWarp0;
+    if ((threadIdx.x & 31) == 0) red[w] = v;
+    named_bar(1, kPrologueThreads);
+    double t = 0.0;
+#pragma unroll
+    for (int i = 0; i < kPrologueThreads / 32; ++i) t += red[i];
+    named_bar(1, kPrologueThreads);
+    return t;
+}
+
 __device__ __forceinline__ int pro_sum(int v, int* red)
 {
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
@@ -157,42 +170,66 @@ __device__ __forceinline__ int pro_sum(int v, int* red)
 }
 
 // Quantise one x row into the resident operand (token m); returns s and the
-// row sum of q.  The arithmetic is bl_quant.cu's: amax over the row (an
-// unsigned max over the bit patterns with the sign cleared -- integer order
-// is numeric order for non-negative IEEE values, and NaN/Inf sort above
-// every finite value, so it also flags non-finite input), s = 127 /
-// max(amax, 1e-5) (IEEE divide), q = rint(x * s) (one round-to-nearest-even
-// conversion: |x * s| < 127.5, so the clamp of the definition never binds).
-template <int MT, typename XT>
-__device__ void quantise_row(const XT* __restrict__ row, int K, int m, uint8_t* bres, int* red, float* s_out,
-                             int* sumq_out, unsigned* status)
+// row sum of q.  The arithmetic is bl_quant.cu's: with a gain vector
+// (SubLN), first ms = sum x^2 / K in fp64, r = fp32(1 / sqrt(ms + eps)) and
+// x <- (x * r) * g in fp32; then amax over the row (an unsigned max over the
+// bit patterns with the sign cleared -- integer order is numeric order for
+// non-negative IEEE values, and NaN/Inf sort above every finite value, so it
+// also flags non-finite input), s = 127 / max(amax, 1e-5) (IEEE divide), q =
+// rint(x * s) (one round-to-nearest-even conversion: |x * s| < 127.5, so the
+// clamp of the definition never binds).
+template <int MT, typename XT, bool NORM>
+__device__ void quantise_row(const XT* __restrict__ row, int K, int m, uint8_t* bres, int* red, double* redd,
+                             const float* __restrict__ gain, double eps, float* s_out, int* sumq_out,
+                             unsigned* status)
 {
     const int tp = threadIdx.x - 32 * kExpWarp0;
     constexpr bool BF16 = sizeof(XT) == 2;
     constexpr int VE = 16 / sizeof(XT);
     const bool vec = (K % VE) == 0;
     const int nv = K / VE;
-    uint32_t mhi = 0, mlo = 0;
     const uint4* rv = reinterpret_cast<const uint4*>(row);
+    auto elem = [&](const uint4& u, int i) -> float {
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+        if constexpr (BF16) return __uint_as_float((i & 1) ? (w[i >> 1] & 0xFFFF0000u) : (w[i >> 1] << 16));
+        return __uint_as_float(w[i]);
+    };
+    float r32 = 1.0f;
+    if constexpr (NORM) {
+        double ss = 0.0;
+        if (vec) {
+            for (int v = tp; v < nv; v += kPrologueThreads) {
+                const uint4 u = __ldg(rv + v);
+#pragma unroll
+                for (int i = 0; i < VE; ++i) {
+                    const double d = (double)elem(u, i);
+                    ss += d * d;
+                }
+            }
+        } else {
+            for (int k = tp; k < K; k += kPrologueThreads) {
+                const double d = (double)to_f(row[k]);
+                ss += d * d;
+            }
+        }
+        ss = pro_sum_f64(ss, redd);
+        r32 = (float)(1.0 / sqrt(ss / (double)K + eps));
+    }
+    auto xn = [&](float v, int k) -> float {
+        if constexpr (NORM) return __fmul_rn(__fmul_rn(v, r32), __ldg(gain + k));
+        return v;
+    };
+    uint32_t mb = 0;
     if (vec) {
         for (int v = tp; v < nv; v += kPrologueThreads) {
             const uint4 u = __ldg(rv + v);
-            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                if constexpr (BF16) {
-                    mhi = max(mhi, w[i] & 0x7FFF0000u);
-                    mlo = max(mlo, (w[i] << 16) & 0x7FFF0000u);
-                } else {
-                    mhi = max(mhi, w[i] & 0x7FFFFFFFu);
-                }
-            }
+            for (int i = 0; i < VE; ++i) mb = max(mb, __float_as_uint(xn(elem(u, i), v * VE + i)) & 0x7FFFFFFFu);
         }
     } else {
-        for (int k = tp; k < K; k += kPrologueThreads)
-            mhi = max(mhi, __float_as_uint(to_f(row[k])) & 0x7FFFFFFFu);
+        for (int k = tp; k < K; k += kPrologueThreads) mb = max(mb, __float_as_uint(xn(to_f(row[k]), k)) & 0x7FFFFFFFu);
     }
-    const uint32_t mbits = pro_max(max(mhi, mlo), red);
+    const uint32_t mbits = pro_max(mb, red);
     if (mbits >= 0x7F800000u && tp == 0) atomicOr(status, kStatusNonfiniteX);
     const float amax = fmaxf(__uint_as_float(mbits), 1e-5f);
     const float s = 127.0f / amax;
@@ -200,27 +237,14 @@ __device__ void quantise_row(const XT* __restrict__ row, int K, int m, uint8_t* 
     if (vec) {
         for (int v = tp; v < nv; v += kPrologueThreads) {
             const uint4 u = __ldg(rv + v);
-            if constexpr (BF16) {
-                const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-                int c[8];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    c[2 * i] = __float2int_rn(__fmul_rn(__uint_as_float(w[i] << 16), s));
-                    c[2 * i + 1] = __float2int_rn(__fmul_rn(__uint_as_float(w[i] & 0xFFFF0000u), s));
-                }
-                const uint32_t p0 = pack4(c[0], c[1], c[2], c[3]);
-                const uint32_t p1 = pack4(c[4], c[5], c[6], c[7]);
-                part = dp4a_ss(p0, 0x01010101u, part);
-                part = dp4a_ss(p1, 0x01010101u, part);
-                *reinterpret_cast<uint32_t*>(bres + bres_offset<MT>(2 * v, m)) = p0;
-                *reinterpret_cast<uint32_t*>(bres + bres_offset<MT>(2 * v + 1, m)) = p1;
-            } else {
-                const uint32_t p0 = pack4(__float2int_rn(__fmul_rn(__uint_as_float(u.x), s)),
-                                          __float2int_rn(__fmul_rn(__uint_as_float(u.y), s)),
-                                          __float2int_rn(__fmul_rn(__uint_as_float(u.z), s)),
-                                          __float2int_rn(__fmul_rn(__uint_as_float(u.w), s)));
-                part = dp4a_ss(p0, 0x01010101u, part);
-                *reinterpret_cast<uint32_t*>(bres + bres_offset<MT>(v, m)) = p0;
+            for (int p = 0; p < VE / 4; ++p) {
+                int c[4];
+#pragma unroll
+                for (int b = 0; b < 4; ++b) c[b] = __float2int_rn(__fmul_rn(xn(elem(u, 4 * p + b), v * VE + 4 * p + b), s));
+                const uint32_t word = pack4(c[0], c[1], c[2], c[3]);
+                part = dp4a_ss(word, 0x01010101u, part);
+                *reinterpret_cast<uint32_t*>(bres + bres_offset<MT>(v * (VE / 4) + p, m)) = word;
             }
         }
     } else {
@@ -229,7 +253,7 @@ __device__ void quantise_row(const XT* __restrict__ row, int K, int m, uint8_t* 
 #pragma unroll
             for (int b = 0; b < 4; ++b) {
                 const int k = 4 * kw + b;
-                c[b] = (k < K) ? __float2int_rn(__fmul_rn(to_f(row[k]), s)) : 0;
+                c[b] = (k < K) ? __float2int_rn(__fmul_rn(xn(to_f(row[k]), k), s)) : 0;
             }
             const uint32_t word = pack4(c[0], c[1], c[2], c[3]);
             part = dp4a_ss(word, 0x01010101u, part);
@@ -243,7 +267,7 @@ __device__ void quantise_row(const XT* __restrict__ row, int K, int m, uint8_t* 
     }
 }
 
-template <int MT, bool FUSED, typename XT, typename YT>
+template <int MT, bool FUSED, typename XT, typename YT, bool NORM>
 __global__ void __launch_bounds__(kThreads, 1) dec_tc_kernel(const __grid_constant__ StreamBatch b, unsigned* status)
 {
     constexpr int S = 16 / MT;      // k-slices per row
@@ -259,6 +283,7 @@ __global__ void __launch_bounds__(kThreads, 1) dec_tc_kernel(const __grid_consta
     __shared__ float s_scale[16];
     __shared__ int s_sumq[16];
     __shared__ int red[kPrologueThreads / 32];
+    __shared__ double redd[kPrologueThreads / 32];
     __shared__ int ep[S > 1 ? 128 * MT : 1];
 
     // 1024-aligned dynamic region: resident B operand, then the two
@@ -370,8 +395,8 @@ __global__ void __launch_bounds__(kThreads, 1) dec_tc_kernel(const __grid_consta
 #pragma unroll 1
         for (int m = 0; m < M; ++m) {
             if constexpr (FUSED) {
-                quantise_row<MT, XT>(static_cast<const XT*>(P.x) + (int64_t)m * K, K, m, bres, red, &s_scale[m],
-                                     &s_sumq[m], status);
+                quantise_row<MT, XT, NORM>(static_cast<const XT*>(P.x) + (int64_t)m * K, K, m, bres, red, redd,
+                                           P.gain, b.eps_norm, &s_scale[m], &s_sumq[m], status);
             } else {
                 const uint4* gq = reinterpret_cast<const uint4*>(P.q + (int64_t)m * Kp);
                 int part = 0;
@@ -548,10 +573,10 @@ __global__ void __launch_bounds__(kThreads, 1) dec_tc_kernel(const __grid_consta
     }
 }
 
-template <int MT, bool FUSED, typename XT, typename YT>
+template <int MT, bool FUSED, typename XT, typename YT, bool NORM>
 cudaError_t launch_t(const StreamBatch& b, int grid, size_t smem, unsigned* status, cudaStream_t st)
 {
-    auto fn = dec_tc_kernel<MT, FUSED, XT, YT>;
+    auto fn = dec_tc_kernel<MT, FUSED, XT, YT, NORM>;
     static bool configured[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -577,16 +602,26 @@ cudaError_t launch_t(const StreamBatch& b, int grid, size_t smem, unsigned* stat
     return cudaGetLastError();
 }
 
+template <bool FUSED, typename XT, typename YT, bool NORM>
+cudaError_t launch_mn(const StreamBatch& b, int MT, int grid, size_t smem, unsigned* status, cudaStream_t st)
+{
+    switch (MT) {
+        case 1: return launch_t<1, FUSED, XT, YT, NORM>(b, grid, smem, status, st);
+        case 2: return launch_t<2, FUSED, XT, YT, NORM>(b, grid, smem, status, st);
+        case 4: return launch_t<4, FUSED, XT, YT, NORM>(b, grid, smem, status, st);
+        case 8: return launch_t<8, FUSED, XT, YT, NORM>(b, grid, smem, status, st);
+        default: return launch_t<16, FUSED, XT, YT, NORM>(b, grid, smem, status, st);
+    }
+}
+
+// The normalising prologue (SubLN) is a separate instantiation.
 template <bool FUSED, typename XT, typename YT>
 cudaError_t launch_m(const StreamBatch& b, int MT, int grid, size_t smem, unsigned* status, cudaStream_t st)
 {
-    switch (MT) {
-        case 1: return launch_t<1, FUSED, XT, YT>(b, grid, smem, status, st);
-        case 2: return launch_t<2, FUSED, XT, YT>(b, grid, smem, status, st);
-        case 4: return launch_t<4, FUSED, XT, YT>(b, grid, smem, status, st);
-        case 8: return launch_t<8, FUSED, XT, YT>(b, grid, smem, status, st);
-        default: return launch_t<16, FUSED, XT, YT>(b, grid, smem, status, st);
+    if constexpr (FUSED) {
+        if (b.p[0].gain) return launch_mn<true, XT, YT, true>(b, MT, grid, smem, status, st);
     }
+    return launch_mn<FUSED, XT, YT, false>(b, MT, grid, smem, status, st);
 }
 
 int job_stages_rt(int MT, int64_t K)

@@ -41,24 +41,18 @@ __device__ __forceinline__ float to_f(__nv_bfloat16 v) { return __bfloat162float
 __device__ __forceinline__ void store_y(float* y, int64_t i, float v) { y[i] = v; }
 __device__ __forceinline__ void store_y(__nv_bfloat16* y, int64_t i, float v) { y[i] = __float2bfloat16_rn(v); }
 
-__device__ __forceinline__ int8_t quant_one(float v, float s)
+// sum over the 224 consumer threads (named barrier 1); fixed order
+__device__ __forceinline__ double consumers_sum_f64(double v, double* red)
 {
-    float r = rintf(__fmul_rn(v, s));
-    r = fminf(fmaxf(r, -127.0f), 127.0f);
-    return (int8_t)(int)r;
-}
-
-// max over the 224 consumer threads (named barrier 1)
-__device__ __forceinline__ float consumers_max(float v, float* red)
-{
-    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
     const int cw = (threadIdx.x >> 5) - 1;
     if ((threadIdx.x & 31) == 0) red[cw] = v;
     named_bar(1, kConsumers);
-    float m = red[0];
+    double t = red[0];
 #pragma unroll
-    for (int w = 1; w < kConsumerWarps; ++w) m = fmaxf(m, red[w]);
-    return m;
+    for (int w = 1; w < kConsumerWarps; ++w) t += red[w];
+    named_bar(1, kConsumers);   // red is reused right after
+    return t;
 }
 
 __device__ __forceinline__ int consumers_sum(int v, int* red)
@@ -93,17 +87,19 @@ __device__ __forceinline__ uint32_t pack4(int a, int b, int c, int d)
 }
 
 // Quantise x row (K elements) into q (Kp bytes) in shared memory; returns s.
-// Same arithmetic as bl_quant.cu: amax over the row, s = 127 / max(amax,
-// 1e-5) (IEEE divide), q = clamp(rint(x * s), -127, 127) in fp32.  Two
-// exact shortcuts: (1) max|x| is taken as an unsigned max over the bit
-// patterns with the sign cleared -- for non-negative IEEE values integer
-// order is numeric order, and NaN/Inf patterns sort above every finite
-// value, so the same max also flags non-finite input; (2) rint + clamp +
-// convert is one round-to-nearest-even conversion, since |x * s| < 127.5
-// for finite x (the clamp can never bind).
-template <typename XT>
-__device__ float quantise_row(const XT* __restrict__ row, int K, int Kp, int8_t* q, int* redi, int* sumq_out,
-                              unsigned* status)
+// Same arithmetic as bl_quant.cu: with a gain vector (SubLN), first
+// ms = sum x^2 / K in fp64, r = fp32(1 / sqrt(ms + eps)) and x <- (x * r) * g
+// in fp32; then amax over the row, s = 127 / max(amax, 1e-5) (IEEE divide),
+// q = clamp(rint(x * s), -127, 127) in fp32.  Two exact shortcuts: (1)
+// max|x| is taken as an unsigned max over the bit patterns with the sign
+// cleared -- for non-negative IEEE values integer order is numeric order,
+// and NaN/Inf patterns sort above every finite value, so the same max also
+// flags non-finite input; (2) rint + clamp + convert is one
+// round-to-nearest-even conversion, since |x * s| < 127.5 for finite x (the
+// clamp can never bind).
+template <typename XT, bool NORM>
+__device__ float quantise_row(const XT* __restrict__ row, int K, int Kp, int8_t* q, int* redi, double* redd,
+                              const float* __restrict__ gain, double eps, int* sumq_out, unsigned* status)
 {
     const int t = threadIdx.x - 32;
     constexpr bool BF16 = sizeof(XT) == 2;
@@ -111,22 +107,8 @@ __device__ float quantise_row(const XT* __restrict__ row, int K, int Kp, int8_t*
     constexpr int VR = 4;                 // vectors a thread keeps in registers
     const int nv = K / VE;
     const bool vec = (K % VE) == 0;
-    const bool held = vec && nv <= VR * kConsumers;   // pass 2 needs no reload
+    const bool held = vec && nv <= VR * kConsumers;   // later passes need no reload
     uint4 keep[VR];
-    uint32_t mbits = 0;                   // max |x| bit pattern (fp32 layout)
-    uint32_t mhi = 0, mlo = 0;
-    auto amax_of = [&](const uint4 u) {
-        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            if constexpr (BF16) {
-                mhi = max(mhi, w[i] & 0x7FFF0000u);
-                mlo = max(mlo, (w[i] << 16) & 0x7FFF0000u);
-            } else {
-                mhi = max(mhi, w[i] & 0x7FFFFFFFu);
-            }
-        }
-    };
     const uint4* rv = reinterpret_cast<const uint4*>(row);
     if (held) {
 #pragma unroll
@@ -134,53 +116,116 @@ __device__ float quantise_row(const XT* __restrict__ row, int K, int Kp, int8_t*
             const int v = t + j * kConsumers;
             keep[j] = v < nv ? __ldg(rv + v) : make_uint4(0, 0, 0, 0);
         }
+    }
+    // f(vector, index) for each of this thread's vectors (static indices
+    // into keep[]: no local memory)
+    auto each = [&](auto&& f) {
+        if (held) {
 #pragma unroll
-        for (int j = 0; j < VR; ++j) amax_of(keep[j]);   // zero padding does not change the max
-        mbits = max(mhi, mlo);
-    } else if (vec) {
-        for (int v = t; v < nv; v += kConsumers) amax_of(__ldg(rv + v));
-        mbits = max(mhi, mlo);
+            for (int j = 0; j < VR; ++j) {
+                const int v = t + j * kConsumers;
+                if (v < nv) f(keep[j], v);
+            }
+        } else {
+            for (int v = t; v < nv; v += kConsumers) f(__ldg(rv + v), v);
+        }
+    };
+    // element i of a vector as fp32 (bf16 widening is exact)
+    auto elem = [&](const uint4& u, int i) -> float {
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+        if constexpr (BF16) return __uint_as_float((i & 1) ? (w[i >> 1] & 0xFFFF0000u) : (w[i >> 1] << 16));
+        return __uint_as_float(w[i]);
+    };
+
+    float r32 = 1.0f;
+    if constexpr (NORM) {
+        double ss = 0.0;
+        if (vec) {
+            each([&](const uint4& u, int) {
+#pragma unroll
+                for (int i = 0; i < VE; ++i) {
+                    const double d = (double)elem(u, i);
+                    ss += d * d;
+                }
+            });
+        } else {
+            for (int k = t; k < K; k += kConsumers) {
+                const double d = (double)to_f(row[k]);
+                ss += d * d;
+            }
+        }
+        ss = consumers_sum_f64(ss, redd);
+        r32 = (float)(1.0 / sqrt(ss / (double)K + eps));
+    }
+    auto xn = [&](float v, int k) -> float {
+        if constexpr (NORM) return __fmul_rn(__fmul_rn(v, r32), __ldg(gain + k));
+        return v;
+    };
+    // the gains of vector v (E floats, 16-byte aligned), loaded together
+    auto gains_of = [&](int v, float (&g)[VE]) {
+        const float4* gp = reinterpret_cast<const float4*>(gain) + v * (VE / 4);
+#pragma unroll
+        for (int p = 0; p < VE / 4; ++p) {
+            const float4 f = __ldg(gp + p);
+            g[4 * p] = f.x;
+            g[4 * p + 1] = f.y;
+            g[4 * p + 2] = f.z;
+            g[4 * p + 3] = f.w;
+        }
+    };
+
+    uint32_t mbits = 0;
+    if (vec) {
+        each([&](const uint4& u, int v) {
+            if constexpr (!NORM) {
+                const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    if constexpr (BF16) {
+                        mbits = max(mbits, w[i] & 0x7FFF0000u);
+                        mbits = max(mbits, (w[i] << 16) & 0x7FFF0000u);
+                    } else {
+                        mbits = max(mbits, w[i] & 0x7FFFFFFFu);
+                    }
+                }
+            } else {
+                float g[VE];
+                gains_of(v, g);
+#pragma unroll
+                for (int i = 0; i < VE; ++i)
+                    mbits = max(mbits, __float_as_uint(__fmul_rn(__fmul_rn(elem(u, i), r32), g[i])) & 0x7FFFFFFFu);
+            }
+        });
     } else {
-        for (int k = t; k < K; k += kConsumers) mbits = max(mbits, __float_as_uint(to_f(row[k])) & 0x7FFFFFFFu);
+        for (int k = t; k < K; k += kConsumers) mbits = max(mbits, __float_as_uint(xn(to_f(row[k]), k)) & 0x7FFFFFFFu);
     }
     mbits = (uint32_t)consumers_max_int((int)mbits, redi);
     if (mbits >= 0x7F800000u && t == 0) atomicOr(status, kStatusNonfiniteX);
     const float amax = fmaxf(__uint_as_float(mbits), 1e-5f);
     const float s = 127.0f / amax;
     int part = 0;
-    auto quant_store = [&](const uint4 u, int v) {
-        if constexpr (BF16) {
-            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-            int c[8];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                c[2 * i] = __float2int_rn(__fmul_rn(__uint_as_float(w[i] << 16), s));
-                c[2 * i + 1] = __float2int_rn(__fmul_rn(__uint_as_float(w[i] & 0xFFFF0000u), s));
-            }
-            const uint32_t p0 = pack4(c[0], c[1], c[2], c[3]);
-            const uint32_t p1 = pack4(c[4], c[5], c[6], c[7]);
-            part = dp4a_ss(p0, 0x01010101u, part);
-            part = dp4a_ss(p1, 0x01010101u, part);
-            *reinterpret_cast<uint2*>(q + v * 8) = make_uint2(p0, p1);
-        } else {
-            const uint32_t p0 = pack4(__float2int_rn(__fmul_rn(__uint_as_float(u.x), s)),
-                                      __float2int_rn(__fmul_rn(__uint_as_float(u.y), s)),
-                                      __float2int_rn(__fmul_rn(__uint_as_float(u.z), s)),
-                                      __float2int_rn(__fmul_rn(__uint_as_float(u.w), s)));
-            part = dp4a_ss(p0, 0x01010101u, part);
-            *reinterpret_cast<uint32_t*>(q + v * 4) = p0;
-        }
-    };
     if (vec) {
-        if (held) {
+        each([&](const uint4& u, int v) {
+            float g[VE];
+            if constexpr (NORM) gains_of(v, g);
+            uint32_t w[VE / 4];
 #pragma unroll
-            for (int j = 0; j < VR; ++j) {
-                const int v = t + j * kConsumers;
-                if (v < nv) quant_store(keep[j], v);
+            for (int p = 0; p < VE / 4; ++p) {
+                int c[4];
+#pragma unroll
+                for (int b = 0; b < 4; ++b) {
+                    float e = elem(u, 4 * p + b);
+                    if constexpr (NORM) e = __fmul_rn(__fmul_rn(e, r32), g[4 * p + b]);
+                    c[b] = __float2int_rn(__fmul_rn(e, s));
+                }
+                w[p] = pack4(c[0], c[1], c[2], c[3]);
+                part = dp4a_ss(w[p], 0x01010101u, part);
             }
-        } else {
-            for (int v = t; v < nv; v += kConsumers) quant_store(__ldg(rv + v), v);
-        }
+            if constexpr (BF16)
+                *reinterpret_cast<uint2*>(q + v * 8) = make_uint2(w[0], w[1]);
+            else
+                *reinterpret_cast<uint32_t*>(q + v * 4) = w[0];
+        });
         for (int k4 = K + 4 * t; k4 < Kp; k4 += 4 * kConsumers) *reinterpret_cast<uint32_t*>(q + k4) = 0u;
     } else {
         for (int k4 = 4 * t; k4 < Kp; k4 += 4 * kConsumers) {
@@ -188,7 +233,7 @@ __device__ float quantise_row(const XT* __restrict__ row, int K, int Kp, int8_t*
 #pragma unroll
             for (int b = 0; b < 4; ++b) {
                 const int k = k4 + b;
-                c[b] = (k < K) ? __float2int_rn(__fmul_rn(to_f(row[k]), s)) : 0;
+                c[b] = (k < K) ? __float2int_rn(__fmul_rn(xn(to_f(row[k]), k), s)) : 0;
             }
             const uint32_t word = pack4(c[0], c[1], c[2], c[3]);
             *reinterpret_cast<uint32_t*>(q + k4) = word;
@@ -221,7 +266,7 @@ __device__ __forceinline__ void dot_chunk(const uint4 wv, const int8_t* qs, int 
     }
 }
 
-template <int MT, bool FUSED, typename XT, typename YT, int MINB>
+template <int MT, bool FUSED, typename XT, typename YT, int MINB, bool NORM>
 __global__ void __launch_bounds__(kThreads, MINB)
 stream_kernel(const __grid_constant__ StreamBatch b, unsigned* status)
 {
@@ -229,7 +274,7 @@ stream_kernel(const __grid_constant__ StreamBatch b, unsigned* status)
     __shared__ uint64_t full_bar[kMaxStages], empty_bar[kMaxStages];
     __shared__ float s_scale[MT];
     __shared__ int s_sumq[MT];
-    __shared__ float redf[kConsumerWarps];
+    __shared__ double redd[kConsumerWarps];
     __shared__ int redi[kConsumerWarps];
     __shared__ int abort_flag;
     __shared__ int piece_ok[2];
@@ -299,7 +344,8 @@ stream_kernel(const __grid_constant__ StreamBatch b, unsigned* status)
 #pragma unroll 1
             for (int m = 0; m < M; ++m) {
                 int sq;
-                const float s = quantise_row<XT>(xb + (int64_t)m * K, K, Kp, qs + m * Kp, redi, &sq, status);
+                const float s = quantise_row<XT, NORM>(xb + (int64_t)m * K, K, Kp, qs + m * Kp, redi, redd,
+                                                       P.gain, b.eps_norm, &sq, status);
                 if (threadIdx.x == 32) {
                     s_scale[m] = s;
                     s_sumq[m] = sq;
@@ -479,10 +525,10 @@ stream_kernel(const __grid_constant__ StreamBatch b, unsigned* status)
     }
 }
 
-template <int MT, bool FUSED, typename XT, typename YT, int MINB>
+template <int MT, bool FUSED, typename XT, typename YT, int MINB, bool NORM>
 cudaError_t launch_t(const StreamBatch& b, int grid, size_t smem, unsigned* status, cudaStream_t st)
 {
-    auto fn = stream_kernel<MT, FUSED, XT, YT, MINB>;
+    auto fn = stream_kernel<MT, FUSED, XT, YT, MINB, NORM>;
     static bool configured[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -512,32 +558,43 @@ cudaError_t launch_t(const StreamBatch& b, int grid, size_t smem, unsigned* stat
     return cudaGetLastError();
 }
 
-template <bool FUSED, typename XT, typename YT, int MINB>
+template <bool FUSED, typename XT, typename YT, int MINB, bool NORM>
 cudaError_t launch_m(const StreamBatch& b, int grid, size_t smem, unsigned* status, cudaStream_t st)
 {
     switch (stream_tokens(b.M)) {
-        case 1: return launch_t<1, FUSED, XT, YT, MINB>(b, grid, smem, status, st);
-        case 2: return launch_t<2, FUSED, XT, YT, MINB>(b, grid, smem, status, st);
-        case 4: return launch_t<4, FUSED, XT, YT, MINB>(b, grid, smem, status, st);
-        case 8: return launch_t<8, FUSED, XT, YT, MINB>(b, grid, smem, status, st);
-        default: return launch_t<16, FUSED, XT, YT, MINB>(b, grid, smem, status, st);
+        case 1: return launch_t<1, FUSED, XT, YT, MINB, NORM>(b, grid, smem, status, st);
+        case 2: return launch_t<2, FUSED, XT, YT, MINB, NORM>(b, grid, smem, status, st);
+        case 4: return launch_t<4, FUSED, XT, YT, MINB, NORM>(b, grid, smem, status, st);
+        case 8: return launch_t<8, FUSED, XT, YT, MINB, NORM>(b, grid, smem, status, st);
+        default: return launch_t<16, FUSED, XT, YT, MINB, NORM>(b, grid, smem, status, st);
     }
 }
 
 // 4 CTAs per SM (64 registers) only for up to 4 tokens; more tokens need
 // the registers of the 2-CTA form.
-template <bool FUSED, typename XT, typename YT>
-cudaError_t launch_b(const StreamBatch& b, int minb, int grid, size_t smem, unsigned* status, cudaStream_t st)
+template <bool FUSED, typename XT, typename YT, bool NORM>
+cudaError_t launch_n(const StreamBatch& b, int minb, int grid, size_t smem, unsigned* status, cudaStream_t st)
 {
     if (minb == 4) {
         switch (stream_tokens(b.M)) {
-            case 1: return launch_t<1, FUSED, XT, YT, 4>(b, grid, smem, status, st);
-            case 2: return launch_t<2, FUSED, XT, YT, 4>(b, grid, smem, status, st);
-            case 4: return launch_t<4, FUSED, XT, YT, 4>(b, grid, smem, status, st);
+            case 1: return launch_t<1, FUSED, XT, YT, 4, NORM>(b, grid, smem, status, st);
+            case 2: return launch_t<2, FUSED, XT, YT, 4, NORM>(b, grid, smem, status, st);
+            case 4: return launch_t<4, FUSED, XT, YT, 4, NORM>(b, grid, smem, status, st);
             default: return cudaErrorNotSupported;
         }
     }
-    return launch_m<FUSED, XT, YT, 2>(b, grid, smem, status, st);
+    return launch_m<FUSED, XT, YT, 2, NORM>(b, grid, smem, status, st);
+}
+
+// The normalising prologue (SubLN) is a separate instantiation, so the
+// plain kernels keep their own register allocation.
+template <bool FUSED, typename XT, typename YT>
+cudaError_t launch_b(const StreamBatch& b, int minb, int grid, size_t smem, unsigned* status, cudaStream_t st)
+{
+    if constexpr (FUSED) {
+        if (b.p[0].gain) return launch_n<true, XT, YT, true>(b, minb, grid, smem, status, st);
+    }
+    return launch_n<FUSED, XT, YT, false>(b, minb, grid, smem, status, st);
 }
 
 }  // namespace

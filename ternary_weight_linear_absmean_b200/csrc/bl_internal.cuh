@@ -43,6 +43,9 @@ int absmean_blocks(int64_t count);
 
 cudaError_t launch_quant(const void* x, bl_dtype xt, int64_t M, int64_t K, int8_t* q, float* s,
                          unsigned* status, cudaStream_t st);
+// SubLN (RMS normalisation with gain [K], epsilon eps) then the quantiser.
+cudaError_t launch_rmsnorm_quant(const void* x, bl_dtype xt, const float* gain, double eps, int64_t M, int64_t K,
+                                 int8_t* q, float* s, unsigned* status, cudaStream_t st);
 
 // One problem of the decode kernel (packed ternary x int8 -> y).
 struct GemvProblem {
@@ -77,6 +80,7 @@ struct StreamProblem {
     const float* gamma32;
     void* y;
     int32_t* acc;           // optional
+    const float* gain;      // fused form: SubLN gain [K] (RMS normalisation before the quantiser), or NULL
     int64_t N, K;
     int cta_begin;          // set by plan_stream
     int ctas;               // set by plan_stream
@@ -91,6 +95,7 @@ struct StreamBatch {
     int stages;             // set by plan_stream
     int q_bytes;            // set by plan_stream
     int layout_tokens;      // tensor-core kernel: token slots of its operand layout
+    double eps_norm;        // SubLN epsilon (problems with a gain)
 };
 constexpr int kMaxStages = 12;
 // dynamic shared memory per CTA for `minb` resident CTAs per SM

@@ -109,3 +109,22 @@ def test_decode_kernel_setting_is_host_only(L):
         assert L.bitlinear_get_decode_kernel() == k
     assert L.bitlinear_set_decode_kernel(7) == bl.BL_ERR_ARG
     assert L.bitlinear_get_decode_kernel() == bl.BL_DECODE_AUTO
+
+
+def test_rmsnorm_entries_reject_bad_arguments(L):
+    f = L.bitlinear_rmsnorm_quant_act
+    assert f(A, bl.BL_BF16, None, 1e-6, 4, 64, A, A, None) == bl.BL_ERR_NULL
+    assert f(A, 9, A, 1e-6, 4, 64, A, A, None) == bl.BL_ERR_DTYPE
+    assert f(A, bl.BL_BF16, A, 1e-6, 0, 64, A, A, None) == bl.BL_ERR_SHAPE
+    assert f(A, bl.BL_BF16, MIS, 1e-6, 4, 64, A, A, None) == bl.BL_ERR_ALIGN
+    assert f(A, bl.BL_BF16, A, -1.0, 4, 64, A, A, None) == bl.BL_ERR_ARG
+    assert f(A, bl.BL_BF16, A, float("inf"), 4, 64, A, A, None) == bl.BL_ERR_ARG
+    g = L.bitlinear_forward_x_rmsnorm_grouped
+    arr = (C.c_void_p * 2)(A, A)
+    i64 = (C.c_int64 * 2)(8, 64)
+    assert g(0, arr, bl.BL_BF16, arr, 1e-6, arr, arr, 1, i64, i64, arr, bl.BL_F32, None) == bl.BL_ERR_ARG
+    assert g(2, arr, bl.BL_BF16, None, 1e-6, arr, arr, 1, i64, i64, arr, bl.BL_F32, None) == bl.BL_ERR_NULL
+    assert g(2, arr, bl.BL_BF16, arr, float("nan"), arr, arr, 1, i64, i64, arr, bl.BL_F32, None) == bl.BL_ERR_ARG
+    assert g(2, arr, bl.BL_BF16, arr, 1e-6, arr, arr, 17, i64, i64, arr, bl.BL_F32, None) == bl.BL_ERR_SHAPE
+    bad = (C.c_void_p * 2)(A, MIS)
+    assert g(2, arr, bl.BL_BF16, bad, 1e-6, arr, arr, 1, i64, i64, arr, bl.BL_F32, None) == bl.BL_ERR_ALIGN
