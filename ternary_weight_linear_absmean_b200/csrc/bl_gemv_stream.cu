@@ -99,7 +99,8 @@ __device__ __forceinline__ uint32_t pack4(int a, int b, int c, int d)
 // clamp can never bind).
 template <typename XT, bool NORM>
 __device__ float quantise_row(const XT* __restrict__ row, int K, int Kp, int8_t* q, int* redi, double* redd,
-                              const float* __restrict__ gain, double eps, int* sumq_out, unsigned* status)
+                              const float* __restrict__ gain, double eps, int* sumq_out, unsigned* status,
+                              bool signal_loads)
 {
     const int t = threadIdx.x - 32;
     constexpr bool BF16 = sizeof(XT) == 2;
@@ -117,6 +118,8 @@ __device__ float quantise_row(const XT* __restrict__ row, int K, int Kp, int8_t*
             keep[j] = v < nv ? __ldg(rv + v) : make_uint4(0, 0, 0, 0);
         }
     }
+    // the loads above are issued: the producer may now queue the weight copies
+    if (signal_loads) named_bar_arrive(4, kThreads);
     // f(vector, index) for each of this thread's vectors (static indices
     // into keep[]: no local memory)
     auto each = [&](auto&& f) {
@@ -277,7 +280,6 @@ stream_kernel(const __grid_constant__ StreamBatch b, unsigned* status)
     __shared__ double redd[kConsumerWarps];
     __shared__ int redi[kConsumerWarps];
     __shared__ int abort_flag;
-    __shared__ int piece_ok[2];
 
     // ---- which problem, which tiles (cheap: the CTA's first copy waits on it)
     int pi = 0;
@@ -326,12 +328,19 @@ stream_kernel(const __grid_constant__ StreamBatch b, unsigned* status)
             prefetch_l2_bulk(src + o, (head - o) < (uint32_t)kStageBytes ? (head - o) : (uint32_t)kStageBytes);
     }
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    if (threadIdx.x == 0) {
-        for (int j = 0; j < first; ++j) {
-            const uint32_t left = range - (uint32_t)j * kStageBytes;
-            const uint32_t len = left < (uint32_t)kStageBytes ? left : (uint32_t)kStageBytes;
-            mbar_arrive_expect_tx(&full_bar[j], len);
-            bulk_g2s(ring + (size_t)j * kStageBytes, src + (int64_t)j * kStageBytes, len, &full_bar[j]);
+    if (warp == 0) {
+        // The consumers' first activation loads go out before the weight
+        // copies: the row is small and on the critical path (quantisation
+        // precedes every product), and behind ~50 KB of copies per CTA it
+        // would wait its turn in the memory system.
+        named_bar(4, kThreads);
+        if (lane == 0) {
+            for (int j = 0; j < first; ++j) {
+                const uint32_t left = range - (uint32_t)j * kStageBytes;
+                const uint32_t len = left < (uint32_t)kStageBytes ? left : (uint32_t)kStageBytes;
+                mbar_arrive_expect_tx(&full_bar[j], len);
+                bulk_g2s(ring + (size_t)j * kStageBytes, src + (int64_t)j * kStageBytes, len, &full_bar[j]);
+            }
         }
     }
 
@@ -345,7 +354,7 @@ stream_kernel(const __grid_constant__ StreamBatch b, unsigned* status)
             for (int m = 0; m < M; ++m) {
                 int sq;
                 const float s = quantise_row<XT, NORM>(xb + (int64_t)m * K, K, Kp, qs + m * Kp, redi, redd,
-                                                       P.gain, b.eps_norm, &sq, status);
+                                                       P.gain, b.eps_norm, &sq, status, m == 0);
                 if (threadIdx.x == 32) {
                     s_scale[m] = s;
                     s_sumq[m] = sq;
@@ -353,6 +362,7 @@ stream_kernel(const __grid_constant__ StreamBatch b, unsigned* status)
                 named_bar(1, kConsumers);
             }
         } else {
+            named_bar_arrive(4, kThreads);
 #pragma unroll 1
             for (int m = 0; m < M; ++m) {
                 const uint4* gq = reinterpret_cast<const uint4*>(P.q + (int64_t)m * Kp);
@@ -434,19 +444,13 @@ stream_kernel(const __grid_constant__ StreamBatch b, unsigned* status)
 #pragma unroll 1
     for (int j = 0; j < npieces; ++j) {
         const int s = j % stages, round = j / stages;
-        // one consumer warp polls the stage barrier; the others sleep in a
-        // hardware named barrier, then confirm the (already complete) phase
-        // themselves, which gives every thread its own acquire of the data.
-        // The outcome is published in piece_ok[j & 1] before the barrier so
-        // that every consumer warp takes the same branch (a warp missing a
-        // later named barrier would leave the others waiting forever).
-        if (cw == 0) {
-            const bool ok = wait_parity(&full_bar[s], round & 1, status, &abort_flag);
-            if (lane == 0) piece_ok[j & 1] = ok && !abort_flag;
-        }
-        named_bar(2, kConsumers);
-        if (!piece_ok[j & 1]) break;
-        mbar_try_wait(&full_bar[s], round & 1);   // completed phase: this thread's acquire
+        // Each consumer warp waits for the stage itself (try_wait suspends
+        // the thread in hardware until the phase completes, and gives every
+        // thread its own acquire of the data); no warp waits for the others.
+        // The verdict is made warp-uniform; the only named barrier after
+        // this loop is reached by every consumer warp exactly once.
+        const bool ok = wait_parity(&full_bar[s], round & 1, status, &abort_flag);
+        if (!__all_sync(0xffffffffu, ok) || abort_flag) break;
         const uint32_t poff = (uint32_t)j * kStageBytes;
         const uint32_t len = (range - poff) < (uint32_t)kStageBytes ? (range - poff) : (uint32_t)kStageBytes;
         const uint8_t* stage = ring + (size_t)s * kStageBytes;

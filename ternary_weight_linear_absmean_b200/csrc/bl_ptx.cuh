@@ -133,6 +133,13 @@ __device__ __forceinline__ void prefetch_tmap(const void* tmap)
 }
 
 // Named barrier over a subset of warps (id 1..15).
+// Arrive at hardware barrier `id` without waiting (the waiting side uses
+// named_bar with the same thread count).
+__device__ __forceinline__ void named_bar_arrive(int id, int threads)
+{
+    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
 __device__ __forceinline__ void named_bar(int id, int threads)
 {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
