@@ -637,8 +637,8 @@ int job_stages_rt(int MT, int64_t K)
 
 }  // namespace
 
-// One CTA per SM.  CTAs go to the problems in proportion to their packed
-// bytes (at least one each, at most one per tile); each CTA gets a
+// One CTA per SM.  CTAs go to the problems by assign_ctas (smallest largest
+// per-CTA share; at least one each, at most one per tile); each CTA gets a
 // contiguous range of whole tiles.  Shared memory: the resident activation
 // operand (MT * Kp bytes, rounded up to whole stages) and two rings of 6
 // (else 4 or 2) 8 KiB stages.  MT (the operand's token slots, >= M) is the
@@ -686,29 +686,10 @@ bool plan_dec_tc(StreamBatch& b, int* grid, size_t* smem)
     }
     if (MT == 0) return false;
     const int64_t rings = 2 * (int64_t)depth * kStage;
-    int assigned = 0;
-    double rem[kMaxGroup];
-    for (int i = 0; i < b.count; ++i) {
-        const int64_t bytes = padded_n(b.p[i].N) * padded_k(b.p[i].K) / 4;
-        const double share = (double)target * (double)bytes / (double)total;
-        int c = (int)share;
-        if (c < 1) c = 1;
-        b.p[i].ctas = c;
-        rem[i] = share - c;
-        assigned += c;
-    }
-    while (assigned < target) {
-        int best = 0;
-        for (int i = 1; i < b.count; ++i)
-            if (rem[i] > rem[best]) best = i;
-        b.p[best].ctas++;
-        rem[best] -= 1.0;
-        assigned++;
-    }
+    if (!assign_ctas(b, target)) return false;
     int begin = 0;
     for (int i = 0; i < b.count; ++i) {
         const int64_t tiles = padded_n(b.p[i].N) / 8;
-        if (b.p[i].ctas > tiles) b.p[i].ctas = (int)tiles;
         b.p[i].cta_begin = begin;
         b.cta_begin[i] = begin;
         b.p[i].tiles_base = (int)(tiles / b.p[i].ctas);

@@ -618,7 +618,40 @@ int sm_count()
     return cached[dev];
 }
 
-// Plans CTAs per problem (proportional to packed bytes) and the shared
+// CTAs per problem so that the largest per-CTA share of packed bytes,
+// ceil(tiles / ctas) * tile bytes, is as small as possible (greedy: the next
+// CTA always goes to the problem whose share is currently largest; one CTA
+// per problem at least, one per tile at most).  Whole tiles per CTA make the
+// granularity coarse for long rows (13.8 KB per tile at K = 6912), so a
+// share proportional to bytes alone can leave one problem's CTAs with 45%
+// more work than the rest.
+bool assign_ctas(StreamBatch& b, int target)
+{
+    if (b.count > target) return false;
+    int64_t tiles[kMaxGroup], tb[kMaxGroup];
+    for (int i = 0; i < b.count; ++i) {
+        tiles[i] = padded_n(b.p[i].N) / 8;
+        tb[i] = tile_bytes(b.p[i].K);
+        b.p[i].ctas = 1;
+    }
+    for (int used = b.count; used < target; ++used) {
+        int best = -1;
+        int64_t worst = -1;
+        for (int i = 0; i < b.count; ++i) {
+            if (b.p[i].ctas >= tiles[i]) continue;
+            const int64_t load = (tiles[i] + b.p[i].ctas - 1) / b.p[i].ctas * tb[i];
+            if (load > worst) {
+                worst = load;
+                best = i;
+            }
+        }
+        if (best < 0) break;
+        b.p[best].ctas++;
+    }
+    return true;
+}
+
+// Plans CTAs per problem (assign_ctas) and the shared
 // memory split for `minb` resident CTAs per SM.  Returns false if the
 // problems do not fit.
 bool plan_stream(StreamBatch& b, int minb, int* grid, size_t* smem)
@@ -632,31 +665,11 @@ bool plan_stream(StreamBatch& b, int minb, int* grid, size_t* smem)
         total += bytes;
         kp_max = kp_max > padded_k(b.p[i].K) ? kp_max : padded_k(b.p[i].K);
     }
-    // CTAs per problem: largest-remainder share of `target`, >= 1, <= tiles
-    int assigned = 0;
-    double rem[kMaxGroup];
-    for (int i = 0; i < b.count; ++i) {
-        const int64_t bytes = padded_n(b.p[i].N) * padded_k(b.p[i].K) / 4;
-        const double share = (double)target * (double)bytes / (double)total;
-        int c = (int)share;
-        if (c < 1) c = 1;
-        b.p[i].ctas = c;
-        rem[i] = share - c;
-        assigned += c;
-    }
-    while (assigned < target) {
-        int best = 0;
-        for (int i = 1; i < b.count; ++i)
-            if (rem[i] > rem[best]) best = i;
-        b.p[best].ctas++;
-        rem[best] -= 1.0;
-        assigned++;
-    }
+    if (!assign_ctas(b, target)) return false;
     int64_t tiles_max = 1;
     int begin = 0;
     for (int i = 0; i < b.count; ++i) {
         const int64_t tiles = padded_n(b.p[i].N) / 8;
-        if (b.p[i].ctas > tiles) b.p[i].ctas = (int)tiles;
         b.p[i].cta_begin = begin;
         b.cta_begin[i] = begin;
         b.p[i].tiles_base = (int)(tiles / b.p[i].ctas);

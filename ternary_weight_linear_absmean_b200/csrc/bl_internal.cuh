@@ -103,6 +103,8 @@ constexpr int stream_budget(int minb) { return minb >= 4 ? 54 * 1024 : 110 * 102
 int stream_tokens(int64_t M);
 int sm_count();
 bool plan_stream(StreamBatch& b, int minb, int* grid, size_t* smem);
+// CTAs per problem (fills p[i].ctas) minimising the largest per-CTA byte share.
+bool assign_ctas(StreamBatch& b, int target);
 // Returns cudaErrorNotSupported if the shapes do not fit (shared memory).
 cudaError_t launch_stream(StreamBatch& b, bool fused, bl_dtype xt, bl_dtype yt, unsigned* status,
                           cudaStream_t st);
