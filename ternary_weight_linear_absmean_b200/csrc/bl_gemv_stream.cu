@@ -463,7 +463,9 @@ stream_kernel(const __grid_constant__ StreamBatch b, unsigned* status)
             uint32_t tile = gsp / spans_per_tile;
             uint32_t gin = gsp - tile * spans_per_tile;       // chunk group within the tile
             const uint8_t* wp = stage + cw * kSpan + lane * 16;
-#pragma unroll 1
+            // two spans per trip: independent dot chains and half the loop
+            // overhead (the tile check stays per span)
+#pragma unroll 2
             for (uint32_t sp = (uint32_t)cw; sp < nsp; sp += kConsumerWarps, wp += kStep) {
                 if ((int)tile != cur) {
                     flush();
