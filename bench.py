@@ -55,7 +55,7 @@ def parse_args():
     ap.add_argument("--mode", choices=["grouped", "fused", "separate"], default="grouped",
                     help="decode: grouped = one launch per step; fused = one launch per linear; "
                          "separate = quantise + product launches per linear")
-    ap.add_argument("--decode-kernel", choices=["auto", "tensor", "dp4a", "tile"], default="auto",
+    ap.add_argument("--decode-kernel", choices=["auto", "tensor", "dp4a", "tile", "lut"], default="auto",
                     help="decode kernel for M <= 16 (bitlinear_set_decode_kernel)")
     ap.add_argument("--rmsnorm", action="store_true",
                     help="decode: fuse SubLN (RMS normalisation with a gain per linear) into the quantiser prologue")
@@ -145,8 +145,7 @@ def decode_bytes(lin, M):
 # entry to None when that kernel changes.
 MEASURED_TRAFFIC = {
     # stream_kernel<1, fused, bf16, fp32, 4>, 2B block, M = 1, grouped launch
-    # (None: the kernel has changed since its last capture)
-    ("block2b", "stream_kernel", 1): None,
+    ("block2b", "stream_kernel", 1): 17_464_832,
 }
 
 
@@ -157,7 +156,8 @@ def decode_kernel_name(args, M=1):
     library's fallbacks)."""
     if args.decode_kernel == "auto":
         return "stream_kernel" if M <= 4 else "dec_tc_kernel"
-    return {"tensor": "dec_tc_kernel", "dp4a": "stream_kernel", "tile": "gemv_kernel"}[args.decode_kernel]
+    return {"tensor": "dec_tc_kernel", "dp4a": "stream_kernel", "tile": "gemv_kernel",
+            "lut": "lut_kernel"}[args.decode_kernel]
 
 
 def max_over_ranks(ms, dist, dev):
@@ -617,7 +617,8 @@ def main():
     _build.build()
     torch.cuda.set_device(local)
     bl.bitlinear_set_decode_kernel({"auto": bl.BL_DECODE_AUTO, "tensor": bl.BL_DECODE_TENSOR,
-                                    "dp4a": bl.BL_DECODE_DP4A, "tile": bl.BL_DECODE_TILE}[args.decode_kernel])
+                                    "dp4a": bl.BL_DECODE_DP4A, "tile": bl.BL_DECODE_TILE,
+                                    "lut": bl.BL_DECODE_LUT}[args.decode_kernel])
     config["decode_kernel"] = args.decode_kernel
     if args.rmsnorm:
         config["subln"] = "RMS normalisation with gain fused into every linear's quantiser prologue"

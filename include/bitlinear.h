@@ -222,12 +222,20 @@ bl_status bitlinear_forward_x_rmsnorm_grouped(int count, const void* const* x, b
  *                     into tensor memory (one CTA per SM)
  *   BL_DECODE_DP4A    persistent streaming kernel, dp4a on the CUDA cores
  *   BL_DECODE_TILE    per-tile kernel (the fallback for the largest shapes)
+ *   BL_DECODE_LUT     table-lookup kernel: per group of four activations,
+ *                     the 16 subset sums; the packed fields' two bit planes
+ *                     index them (aratech.ae, "How BitNet.cpp achieves its
+ *                     speed"; devtrends.ru, "How does it work?": lookup
+ *                     tables instead of matrix multiplications).  Only
+ *                     bitlinear_forward with M = 1 and 8 * Kp <= ~196 KiB;
+ *                     the fused calls return BL_ERR_SHAPE under it.  An A/B
+ *                     counterpart: AUTO never selects it.
  * A forced TENSOR or DP4A choice that does not fit the shapes makes the
  * forward calls return BL_ERR_SHAPE.  bitlinear_set_decode_kernel returns
  * BL_OK, or BL_ERR_ARG for an unknown value.  The pages define no such
  * setting: it selects between implementations of the same product.
  * ---------------------------------------------------------------------- */
-enum { BL_DECODE_AUTO = 0, BL_DECODE_TENSOR = 1, BL_DECODE_DP4A = 2, BL_DECODE_TILE = 3 };
+enum { BL_DECODE_AUTO = 0, BL_DECODE_TENSOR = 1, BL_DECODE_DP4A = 2, BL_DECODE_TILE = 3, BL_DECODE_LUT = 4 };
 int bitlinear_set_decode_kernel(int kind);
 int bitlinear_get_decode_kernel(void);
 

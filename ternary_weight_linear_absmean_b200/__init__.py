@@ -20,7 +20,7 @@ LIB_PATH = os.path.join(HERE, "libbitlinear.so")
 BL_OK, BL_ERR_NULL, BL_ERR_SHAPE, BL_ERR_ALIGN, BL_ERR_DTYPE = 0, 1, 2, 3, 4
 BL_ERR_WORKSPACE, BL_ERR_OVERFLOW, BL_ERR_NONFINITE, BL_ERR_CUDA, BL_ERR_ARG, BL_ERR_TIMEOUT = 5, 6, 7, 8, 9, 10
 BL_F32, BL_BF16 = 0, 1
-BL_DECODE_AUTO, BL_DECODE_TENSOR, BL_DECODE_DP4A, BL_DECODE_TILE = 0, 1, 2, 3
+BL_DECODE_AUTO, BL_DECODE_TENSOR, BL_DECODE_DP4A, BL_DECODE_TILE, BL_DECODE_LUT = 0, 1, 2, 3, 4
 
 # Every symbol include/bitlinear.h declares, with (restype, argtypes).
 _vp, _i64, _i32 = C.c_void_p, C.c_int64, C.c_int

@@ -34,6 +34,7 @@ bl_status dispatch_decode(bl::StreamBatch& sb, bool fused, bl_dtype xt, bl_dtype
 {
     const int kind = g_decode_kernel.load();
     if (kind == BL_DECODE_TILE) return kTryNext;
+    if (kind == BL_DECODE_LUT) return BL_ERR_SHAPE;   // unfused form only
     const bool tensor_first = kind == BL_DECODE_TENSOR || (kind == BL_DECODE_AUTO && sb.M > 4);
     for (int pass = 0; pass < 2; ++pass) {
         const bool tensor = (pass == 0) == tensor_first;
@@ -167,6 +168,11 @@ bl_status bitlinear_forward(const int8_t* q, const float* s, const uint8_t* pack
         return bl::launch_gemm_tc(q, s, packed, gamma32, M, N, K, y, yt, acc_debug, status, cs) == cudaSuccess
                    ? BL_OK
                    : BL_ERR_CUDA;
+    if (g_decode_kernel.load() == BL_DECODE_LUT) {
+        if (!bl::lut_supported(M, K)) return BL_ERR_SHAPE;
+        const cudaError_t e = bl::launch_lut(q, s, packed, gamma32, N, K, y, yt, acc_debug, cs);
+        return e == cudaSuccess ? BL_OK : e == cudaErrorNotSupported ? BL_ERR_SHAPE : BL_ERR_CUDA;
+    }
     if (M <= bl::kFusedMaxM) {
         bl::StreamBatch sb;
         std::memset(&sb, 0, sizeof(sb));
@@ -250,7 +256,7 @@ bl_status bitlinear_forward_x_grouped(int count, const void* const* x, bl_dtype 
 
 int bitlinear_set_decode_kernel(int kind)
 {
-    if (kind < BL_DECODE_AUTO || kind > BL_DECODE_TILE) return BL_ERR_ARG;
+    if (kind < BL_DECODE_AUTO || kind > BL_DECODE_LUT) return BL_ERR_ARG;
     g_decode_kernel.store(kind);
     return BL_OK;
 }

@@ -116,6 +116,11 @@ bool plan_dec_tc(StreamBatch& b, int* grid, size_t* smem);
 cudaError_t launch_dec_tc(StreamBatch& b, bool fused, bl_dtype xt, bl_dtype yt, unsigned* status,
                           cudaStream_t st);
 
+// Table-lookup decode kernel (bl_gemv_lut.cu): M = 1, q and s given.
+bool lut_supported(int64_t M, int64_t K);
+cudaError_t launch_lut(const int8_t* q, const float* s, const uint8_t* packed, const float* gamma32, int64_t N,
+                       int64_t K, void* y, bl_dtype yt, int32_t* acc, cudaStream_t st);
+
 // Prefill tensor-core GEMM (tcgen05 kind::i8).  Returns cudaErrorNotSupported
 // when the shape is outside what the kernel handles; the caller then uses
 // the decode kernel.

@@ -104,7 +104,7 @@ def test_forward_x_rejects_bad_arguments(L):
 def test_decode_kernel_setting_is_host_only(L):
     # process-wide choice; no CUDA call behind it
     assert L.bitlinear_get_decode_kernel() == bl.BL_DECODE_AUTO
-    for k in (bl.BL_DECODE_TENSOR, bl.BL_DECODE_DP4A, bl.BL_DECODE_TILE, bl.BL_DECODE_AUTO):
+    for k in (bl.BL_DECODE_TENSOR, bl.BL_DECODE_DP4A, bl.BL_DECODE_TILE, bl.BL_DECODE_LUT, bl.BL_DECODE_AUTO):
         assert L.bitlinear_set_decode_kernel(k) == bl.BL_OK
         assert L.bitlinear_get_decode_kernel() == k
     assert L.bitlinear_set_decode_kernel(7) == bl.BL_ERR_ARG

@@ -113,7 +113,7 @@ def test_grouped(bl, kind, M):
 
 
 def test_set_decode_kernel_rejects_unknown(bl):
-    assert bl.lib().bitlinear_set_decode_kernel(4) == bl.BL_ERR_ARG
+    assert bl.lib().bitlinear_set_decode_kernel(5) == bl.BL_ERR_ARG
     assert bl.lib().bitlinear_set_decode_kernel(-1) == bl.BL_ERR_ARG
     assert bl.bitlinear_get_decode_kernel() == bl.BL_DECODE_AUTO
 
@@ -138,3 +138,48 @@ def test_tensor_kernel_large_operand(bl, M, K):
     assert bl.bitlinear_get_status() == bl.BL_OK
     assert np.array_equal(acc.cpu().numpy(), ref["acc"])
     P.check_y_f32(y.cpu().numpy(), ref["y"], exact=True)
+
+
+@pytest.mark.parametrize("N,K", [(13, 200), (300, 1000), (33, 4097), (2560, 640), (640, 2560), (6912, 2560),
+                                 (2560, 6912), (20000, 64)])
+def test_lut_kernel(bl, N, K):
+    # table-lookup decode (M = 1, unfused form) against the oracle
+    import torch
+    W = synth.weights(N, K, seed=N + 7 * K)
+    x = synth.activations(1, K, seed=K, dtype="bf16", outlier_frac=0.01)
+    ref = oracle.bitlinear(W, x, "bf16")
+    packed, _, g32 = _packed(bl, W)
+    q, s = bl.quant_act(P.to_dev_bf16(x))
+    bl.bitlinear_set_decode_kernel(bl.BL_DECODE_LUT)
+    try:
+        y, acc = bl.forward(q, s, packed, g32, N, K, acc_debug=True)
+        torch.cuda.synchronize()
+    finally:
+        bl.bitlinear_set_decode_kernel(bl.BL_DECODE_AUTO)
+    assert bl.bitlinear_get_status() == bl.BL_OK
+    assert np.array_equal(acc.cpu().numpy(), ref["acc"])
+    P.check_y_f32(y.cpu().numpy(), ref["y"], exact=True)
+
+
+def test_lut_kernel_limits(bl):
+    # M > 1, tables beyond shared memory, and the fused calls are refused
+    import torch
+    W = synth.weights(64, 256, seed=1)
+    packed, _, g32 = _packed(bl, W)
+    x2 = P.to_dev_bf16(synth.activations(2, 256, seed=2, dtype="bf16"))
+    q2, s2 = bl.quant_act(x2)
+    big = torch.zeros((1, 28672), dtype=torch.bfloat16, device="cuda")
+    Wb = torch.zeros((8, 28672), dtype=torch.float32, device="cuda")
+    pb, _, gb = bl.pack(Wb)
+    qb, sb = bl.quant_act(big)
+    bl.bitlinear_set_decode_kernel(bl.BL_DECODE_LUT)
+    try:
+        with pytest.raises(bl.BitLinearError):
+            bl.forward(q2, s2, packed, g32, 64, 256)
+        with pytest.raises(bl.BitLinearError):
+            bl.forward(qb, sb, pb, gb, 8, 28672)
+        with pytest.raises(bl.BitLinearError):
+            bl.forward_x(x2[:1], packed, g32, 64, 256)
+    finally:
+        bl.bitlinear_set_decode_kernel(bl.BL_DECODE_AUTO)
+    torch.cuda.synchronize()
