@@ -145,7 +145,10 @@ def decode_bytes(lin, M):
 # entry to None when that kernel changes.
 MEASURED_TRAFFIC = {
     # stream_kernel<1, fused, bf16, fp32, 4>, 2B block, M = 1, grouped launch
-    ("block2b", "stream_kernel", 1): 17_464_832,
+    ("block2b", "stream_kernel", 1): 17_471_744,
+    # gemm_tc_kernel<bf16>, M = 2048: mean of the step's two launches
+    # (2560->6912: 9,722,368 B; 6912->2560: 18,645,504 B)
+    ("prefill", "gemm_tc_kernel", 2048): 14_183_936,
 }
 
 
@@ -496,7 +499,8 @@ def run_prefill(torch, bl, args, dev, stream, dist, l2, steps):
             "value": ops / (ms / steps / 1e3) / 1e12, "unit": "TOPS", "ms_per_step": ms / steps,
             "steps": steps, "launches_per_step": 2 * len(lin),
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": int8_peak, "unit": "TFLOP/s",
-                         "frac": achieved / int8_peak, "traffic": None,
+                         "frac": achieved / int8_peak,
+                         "traffic": MEASURED_TRAFFIC.get(("prefill", "gemm_tc_kernel", M)),
                          "kernel": "gemm_tc_kernel (tcgen05 kind::i8, weights expanded into TMEM)",
                          "peak_kind": f"{peaks['kind']} bf16 burst x nominal int8/bf16 ratio 2",
                          "avg_launch_us": kms / steps / len(lin) * 1e3,
