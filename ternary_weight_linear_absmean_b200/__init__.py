@@ -199,6 +199,29 @@ def bitlinear_forward_x_rmsnorm_grouped(xs, gains, eps, packeds, gammas, Ns, Ks,
     _check(st, "bitlinear_forward_x_rmsnorm_grouped")
 
 
+class GroupedDecode:
+    """A prepared bitlinear_forward_x_grouped call: the pointer and size
+    arrays are marshalled once, so each call costs one C call (for decode
+    loops that run the same layers every token).  The tensors must stay
+    alive and in place while the object is used."""
+
+    def __init__(self, xs, packeds, gammas, Ns, Ks, ys):
+        n = len(xs)
+        if not (len(packeds) == len(gammas) == len(Ns) == len(Ks) == len(ys) == n):
+            raise ValueError("grouped arguments must all have the same length")
+        arr_p = C.c_void_p * n
+        arr_i = C.c_int64 * n
+        self._keep = (list(xs), list(packeds), list(gammas), list(ys))
+        self._args = (n, arr_p(*[_dptr(t, "x") for t in xs]), _dtype_code(xs[0].dtype),
+                      arr_p(*[_dptr(t, "packed") for t in packeds]), arr_p(*[_dptr(t, "gamma32") for t in gammas]),
+                      xs[0].shape[0], arr_i(*Ns), arr_i(*Ks), arr_p(*[_dptr(t, "y") for t in ys]),
+                      _dtype_code(ys[0].dtype))
+        self._fn = lib().bitlinear_forward_x_grouped
+
+    def __call__(self, stream=None) -> None:
+        _check(self._fn(*self._args, _stream(stream)), "bitlinear_forward_x_grouped")
+
+
 def bitlinear_get_status(stream=None) -> int:
     return int(lib().bitlinear_get_status(_stream(stream)))
 

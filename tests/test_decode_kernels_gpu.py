@@ -183,3 +183,27 @@ def test_lut_kernel_limits(bl):
     finally:
         bl.bitlinear_set_decode_kernel(bl.BL_DECODE_AUTO)
     torch.cuda.synchronize()
+
+
+def test_prepared_grouped_call_matches_direct_call(bl):
+    # GroupedDecode marshals once; its results equal the plain grouped call's
+    import torch
+    shapes = [(640, 2560), (96, 4097), (300, 1000)]
+    xs, ps, gs, y1, y2 = [], [], [], [], []
+    for i, (N, K) in enumerate(shapes):
+        W = synth.weights(N, K, seed=400 + i)
+        x = synth.activations(1, K, seed=500 + i, dtype="bf16")
+        p, _, g = _packed(bl, W)
+        xs.append(P.to_dev_bf16(x))
+        ps.append(p)
+        gs.append(g)
+        y1.append(torch.empty((1, N), dtype=torch.float32, device="cuda"))
+        y2.append(torch.empty((1, N), dtype=torch.float32, device="cuda"))
+    Ns, Ks = [s[0] for s in shapes], [s[1] for s in shapes]
+    call = bl.GroupedDecode(xs, ps, gs, Ns, Ks, y1)
+    call()
+    call()
+    bl.bitlinear_forward_x_grouped(xs, ps, gs, Ns, Ks, y2)
+    torch.cuda.synchronize()
+    for a, b in zip(y1, y2):
+        assert np.array_equal(a.cpu().numpy(), b.cpu().numpy())
