@@ -16,7 +16,7 @@
  *             each multiply into add / subtract / skip) and sec. 4.1 (2 bits
  *             per weight, packed for wide loads).
  *
- * Readings taken where the pages are silent (each also listed in the design doc):
+ * Readings taken where the pages are silent:
  *   R1  eps = 1e-5 (caller-chosen), added to gamma in fp64, used only for the
  *       codes; the rescale uses gamma itself.
  *   R2  "round" is IEEE round-half-to-even (rint).

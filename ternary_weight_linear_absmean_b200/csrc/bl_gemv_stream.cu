@@ -4,24 +4,29 @@
 // an activation; aratech.ae "BitLinear: the building block" for the int8
 // per-token activations).
 //
-// Launch: two CTAs per SM.  CTAs are shared out among the problems of the
-// launch in proportion to their packed bytes, and each CTA owns a contiguous
-// range of whole 8-row tiles of one problem -- in the packed layout that is
-// one contiguous byte range.
+// Launch: 4 CTAs per SM (up to 4 tokens; 2 above), with programmatic
+// dependent launch.  CTAs are shared out among the problems of the launch so
+// that the largest per-CTA share of whole tiles is as small as possible
+// (assign_ctas), and each CTA owns a contiguous range of whole 8-row tiles of
+// one problem -- in the packed layout that is one contiguous byte range.
 //
 // Inside a CTA (8 warps):
-//   warp 0, lane 0  producer: streams the range into a ring of 16 KiB shared
-//                   memory stages with 1-D bulk copies (cp.async.bulk), one
-//                   mbarrier pair (full/empty) per stage;
+//   warp 0, lane 0  producer (long ranges): streams the range into a ring of
+//                   16 KiB shared-memory stages with 1-D bulk copies
+//                   (cp.async.bulk), one mbarrier pair (full/empty) per
+//                   stage; it issues its first copies only after the
+//                   consumers have issued their activation loads.
 //   warps 1..7      consumers: first quantise x into shared memory (fused
-//                   form) or copy q there, while the first stages are in
-//                   flight; then for each stage take 512-byte spans (4 chunks
-//                   x 8 rows of a tile) round-robin, lane l reading 16 bytes,
-//                   row r = l % 8, and accumulate with dp4a (decode as in
-//                   bl_gemv.cu).  Per-lane partial sums are added into a
-//                   per-(tile, row, token) int32 array in shared memory
-//                   (integer adds: exact and order-independent) whenever the
-//                   lane's tile changes.
+//                   form, optionally with SubLN) or copy q there; then take
+//                   512-byte spans (4 chunks x 8 rows of a tile) round-robin,
+//                   lane l reading 16 bytes, row r = l % 8, and accumulate
+//                   with dp4a (decode as in bl_gemv.cu).  Short ranges
+//                   (<= 128 KiB) skip the ring: the consumers read their
+//                   spans straight from global memory, four in flight per
+//                   lane.  Per-lane partial sums are added into a per-(tile,
+//                   row, token) int32 array in shared memory (integer adds:
+//                   exact and order-independent) whenever the lane's tile
+//                   changes.
 //   epilogue        y = (float)((double)acc * (double)gamma32 / (double)s_m),
 //                   bit-identical to the oracle's rescale.
 #include "bl_internal.cuh"
@@ -304,7 +309,6 @@ stream_kernel(const __grid_constant__ StreamBatch b, unsigned* status)
     const int ci = (int)blockIdx.x - P.cta_begin;
     const int64_t t0 = (int64_t)ci * P.tiles_base + (ci < P.tiles_extra ? ci : P.tiles_extra);
     const int ntl = P.tiles_base + (ci < P.tiles_extra ? 1 : 0);
-    const int64_t t1 = t0 + ntl;
     const uint32_t range = (uint32_t)ntl * TB;                    // < 2^31 (host-checked)
     const uint8_t* src = P.packed + t0 * (int64_t)TB;
     const int stages = b.stages;
