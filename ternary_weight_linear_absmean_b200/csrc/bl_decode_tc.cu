@@ -52,7 +52,8 @@
 //   warps 4-11   expansion, two groups of four taking alternate stages, each
 //                with its own ring of prefetched stages
 //   warps 12-15  epilogue: tcgen05.ld, plane and slice sums, rescale, store
-//   warps 4-15 also quantise x (fused form) or copy q (unfused) first.
+//   warps 4-15 also quantise x (fused form) or copy q (unfused) first, all
+//                token rows together (bl_quant_rows.cuh).
 // Tensor memory (512 columns): five 64-column A stages, three 64-column
 // accumulator sets (4 planes x N = 16), so three jobs can be in flight --
 // decode jobs are short (one or a few stages).
@@ -61,6 +62,7 @@
 #include "bl_internal.cuh"
 #include "bl_ptx.cuh"
 #include "bl_tc.cuh"
+#include "bl_quant_rows.cuh"
 
 namespace bl {
 namespace {
@@ -114,158 +116,8 @@ __host__ __device__ __forceinline__ int job_stages(int64_t K)
     return (int)((chunks_per_row(K) + 4 * S - 1) / (4 * S));
 }
 
-template <typename T>
-__device__ __forceinline__ float to_f(T v);
-template <>
-__device__ __forceinline__ float to_f<float>(float v) { return v; }
-template <>
-__device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 v) { return __bfloat162float(v); }
-
 __device__ __forceinline__ void store_y(float* y, int64_t i, float v) { y[i] = v; }
 __device__ __forceinline__ void store_y(__nv_bfloat16* y, int64_t i, float v) { y[i] = __float2bfloat16_rn(v); }
-
-__device__ __forceinline__ uint32_t pack4(int a, int b, int c, int d)
-{
-    return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
-}
-
-// reductions over the prologue threads (warps 4..15), named barrier 1
-__device__ __forceinline__ uint32_t pro_max(uint32_t v, int* red)
-{
-    for (int o = 16; o > 0; o >>= 1) v = max(v, __shfl_xor_sync(0xffffffffu, v, o));
-    const int w = (threadIdx.x >> 5) - kExpWarp0;
-    if ((threadIdx.x & 31) == 0) red[w] = (int)v;
-    named_bar(1, kPrologueThreads);
-    uint32_t m = (uint32_t)red[0];
-#pragma unroll
-    for (int i = 1; i < kPrologueThreads / 32; ++i) m = max(m, (uint32_t)red[i]);
-    named_bar(1, kPrologueThreads);
-    return m;
-}
-
-__device__ __forceinline__ double pro_sum_f64(double v, double* red)
-{
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    const int w = (threadIdx.x >> 5) - kExpWarp0;
-    if ((threadIdx.x & 31) == 0) red[w] = v;
-    named_bar(1, kPrologueThreads);
-    double t = 0.0;
-#pragma unroll
-    for (int i = 0; i < kPrologueThreads / 32; ++i) t += red[i];
-    named_bar(1, kPrologueThreads);
-    return t;
-}
-
-__device__ __forceinline__ int pro_sum(int v, int* red)
-{
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    const int w = (threadIdx.x >> 5) - kExpWarp0;
-    if ((threadIdx.x & 31) == 0) red[w] = v;
-    named_bar(1, kPrologueThreads);
-    int t = 0;
-#pragma unroll
-    for (int i = 0; i < kPrologueThreads / 32; ++i) t += red[i];
-    named_bar(1, kPrologueThreads);
-    return t;
-}
-
-// Quantise one x row into the resident operand (token m); returns s and the
-// row sum of q.  The arithmetic is bl_quant.cu's: with a gain vector
-// (SubLN), first ms = sum x^2 / K in fp64, r = fp32(1 / sqrt(ms + eps)) and
-// x <- (x * r) * g in fp32; then amax over the row (an unsigned max over the
-// bit patterns with the sign cleared -- integer order is numeric order for
-// non-negative IEEE values, and NaN/Inf sort above every finite value, so it
-// also flags non-finite input), s = 127 / max(amax, 1e-5) (IEEE divide), q =
-// rint(x * s) (one round-to-nearest-even conversion: |x * s| < 127.5, so the
-// clamp of the definition never binds).
-template <int MT, typename XT, bool NORM>
-__device__ void quantise_row(const XT* __restrict__ row, int K, int m, uint8_t* bres, int* red, double* redd,
-                             const float* __restrict__ gain, double eps, float* s_out, int* sumq_out,
-                             unsigned* status)
-{
-    const int tp = threadIdx.x - 32 * kExpWarp0;
-    constexpr bool BF16 = sizeof(XT) == 2;
-    constexpr int VE = 16 / sizeof(XT);
-    const bool vec = (K % VE) == 0;
-    const int nv = K / VE;
-    const uint4* rv = reinterpret_cast<const uint4*>(row);
-    auto elem = [&](const uint4& u, int i) -> float {
-        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-        if constexpr (BF16) return __uint_as_float((i & 1) ? (w[i >> 1] & 0xFFFF0000u) : (w[i >> 1] << 16));
-        return __uint_as_float(w[i]);
-    };
-    float r32 = 1.0f;
-    if constexpr (NORM) {
-        double ss = 0.0;
-        if (vec) {
-            for (int v = tp; v < nv; v += kPrologueThreads) {
-                const uint4 u = __ldg(rv + v);
-#pragma unroll
-                for (int i = 0; i < VE; ++i) {
-                    const double d = (double)elem(u, i);
-                    ss += d * d;
-                }
-            }
-        } else {
-            for (int k = tp; k < K; k += kPrologueThreads) {
-                const double d = (double)to_f(row[k]);
-                ss += d * d;
-            }
-        }
-        ss = pro_sum_f64(ss, redd);
-        r32 = (float)(1.0 / sqrt(ss / (double)K + eps));
-    }
-    auto xn = [&](float v, int k) -> float {
-        if constexpr (NORM) return __fmul_rn(__fmul_rn(v, r32), __ldg(gain + k));
-        return v;
-    };
-    uint32_t mb = 0;
-    if (vec) {
-        for (int v = tp; v < nv; v += kPrologueThreads) {
-            const uint4 u = __ldg(rv + v);
-#pragma unroll
-            for (int i = 0; i < VE; ++i) mb = max(mb, __float_as_uint(xn(elem(u, i), v * VE + i)) & 0x7FFFFFFFu);
-        }
-    } else {
-        for (int k = tp; k < K; k += kPrologueThreads) mb = max(mb, __float_as_uint(xn(to_f(row[k]), k)) & 0x7FFFFFFFu);
-    }
-    const uint32_t mbits = pro_max(mb, red);
-    if (mbits >= 0x7F800000u && tp == 0) atomicOr(status, kStatusNonfiniteX);
-    const float amax = fmaxf(__uint_as_float(mbits), 1e-5f);
-    const float s = 127.0f / amax;
-    int part = 0;
-    if (vec) {
-        for (int v = tp; v < nv; v += kPrologueThreads) {
-            const uint4 u = __ldg(rv + v);
-#pragma unroll
-            for (int p = 0; p < VE / 4; ++p) {
-                int c[4];
-#pragma unroll
-                for (int b = 0; b < 4; ++b) c[b] = __float2int_rn(__fmul_rn(xn(elem(u, 4 * p + b), v * VE + 4 * p + b), s));
-                const uint32_t word = pack4(c[0], c[1], c[2], c[3]);
-                part = dp4a_ss(word, 0x01010101u, part);
-                *reinterpret_cast<uint32_t*>(bres + bres_offset<MT>(v * (VE / 4) + p, m)) = word;
-            }
-        }
-    } else {
-        for (int kw = tp; kw < (K + 3) / 4; kw += kPrologueThreads) {
-            int c[4];
-#pragma unroll
-            for (int b = 0; b < 4; ++b) {
-                const int k = 4 * kw + b;
-                c[b] = (k < K) ? __float2int_rn(__fmul_rn(xn(to_f(row[k]), k), s)) : 0;
-            }
-            const uint32_t word = pack4(c[0], c[1], c[2], c[3]);
-            part = dp4a_ss(word, 0x01010101u, part);
-            *reinterpret_cast<uint32_t*>(bres + bres_offset<MT>(kw, m)) = word;
-        }
-    }
-    const int sq = pro_sum(part, red);
-    if (tp == 0) {
-        *s_out = s;
-        *sumq_out = sq;
-    }
-}
 
 template <int MT, bool FUSED, typename XT, typename YT, bool NORM>
 __global__ void __launch_bounds__(kThreads, 1) dec_tc_kernel(const __grid_constant__ StreamBatch b, unsigned* status)
@@ -282,9 +134,9 @@ __global__ void __launch_bounds__(kThreads, 1) dec_tc_kernel(const __grid_consta
     __shared__ int epi_ok;
     __shared__ float s_scale[16];
     __shared__ int s_sumq[16];
-    __shared__ int red[kPrologueThreads / 32];
-    __shared__ double redd[kPrologueThreads / 32];
     __shared__ int ep[S > 1 ? 128 * MT : 1];
+    __shared__ QuantRowsShared qsh;
+    __shared__ double ss_rows[NORM ? kPrologueThreads / 32 * 16 : 1];
 
     // 1024-aligned dynamic region: resident B operand, then the two
     // expansion groups' rings of D prefetched stages each
@@ -392,29 +244,16 @@ __global__ void __launch_bounds__(kThreads, 1) dec_tc_kernel(const __grid_consta
             *reinterpret_cast<uint4*>(bres + o) = make_uint4(0, 0, 0, 0);
         named_bar(1, kPrologueThreads);
         const int M = b.M;
-#pragma unroll 1
-        for (int m = 0; m < M; ++m) {
-            if constexpr (FUSED) {
-                quantise_row<MT, XT, NORM>(static_cast<const XT*>(P.x) + (int64_t)m * K, K, m, bres, red, redd,
-                                           P.gain, b.eps_norm, &s_scale[m], &s_sumq[m], status);
-            } else {
-                const uint4* gq = reinterpret_cast<const uint4*>(P.q + (int64_t)m * Kp);
-                int part = 0;
-                for (int v = tp; v < Kp / 16; v += kPrologueThreads) {
-                    const uint4 u = __ldg(gq + v);
-                    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        part = dp4a_ss(w[i], 0x01010101u, part);
-                        *reinterpret_cast<uint32_t*>(bres + bres_offset<MT>(4 * v + i, m)) = w[i];
-                    }
-                }
-                const int sq = pro_sum(part, red);
-                if (tp == 0) {
-                    s_scale[m] = P.s[m];
-                    s_sumq[m] = sq;
-                }
-            }
+        auto store_b = [&](int m, int kw, uint32_t w) {
+            *reinterpret_cast<uint32_t*>(bres + bres_offset<MT>(kw, m)) = w;
+        };
+        auto sync_pro = [&]() { named_bar(1, kPrologueThreads); };
+        if constexpr (FUSED) {
+            quantise_rows<MT, kPrologueThreads, XT, NORM>(static_cast<const XT*>(P.x), M, K, P.gain, b.eps_norm, tp,
+                                                          qsh, ss_rows, s_scale, s_sumq, store_b, sync_pro, status);
+        } else {
+            copy_q_rows<MT, kPrologueThreads>(P.q, M, Kp, tp, qsh, s_sumq, store_b, sync_pro);
+            if (tp < M) s_scale[tp] = P.s[tp];
         }
         // generic-proxy writes of the operand, read next by the tensor cores
         fence_proxy_async_smem();

@@ -31,6 +31,7 @@
 //                   bit-identical to the oracle's rescale.
 #include "bl_internal.cuh"
 #include "bl_ptx.cuh"
+#include "bl_quant_rows.cuh"
 
 namespace bl {
 namespace {
@@ -296,6 +297,8 @@ stream_kernel(const __grid_constant__ StreamBatch b, unsigned* status)
     __shared__ double redd[kConsumerWarps];
     __shared__ int redi[kConsumerWarps];
     __shared__ int abort_flag;
+    __shared__ QuantRowsShared qsh;
+    __shared__ double ss_rows[NORM && MT > 1 ? kConsumerWarps * 16 : 1];
 
     // ---- which problem, which tiles (cheap: the CTA's first copy waits on it)
     int pi = 0;
@@ -370,41 +373,30 @@ stream_kernel(const __grid_constant__ StreamBatch b, unsigned* status)
     if (warp != 0) {
         // ------------------------------------------- consumers: prologue
         for (int i = threadIdx.x - 32; i < ntl * 8 * MT; i += kConsumers) sacc[i] = 0;
-        if constexpr (FUSED) {
-            const XT* xb = static_cast<const XT*>(P.x);
-#pragma unroll 1
-            for (int m = 0; m < M; ++m) {
-                int sq;
-                const float s = quantise_row<XT, NORM>(xb + (int64_t)m * K, K, Kp, qs + m * Kp, redi, redd,
-                                                       P.gain, b.eps_norm, &sq, status, m == 0);
-                if (threadIdx.x == 32) {
-                    s_scale[m] = s;
-                    s_sumq[m] = sq;
-                }
-                named_bar(1, kConsumers);
+        const int tp = threadIdx.x - 32;
+        auto store_q = [&](int m, int kw, uint32_t w) { *reinterpret_cast<uint32_t*>(qs + m * Kp + 4 * kw) = w; };
+        auto sync_consumers = [&]() { named_bar(1, kConsumers); };
+        if constexpr (FUSED && MT == 1) {
+            int sq;
+            const float s = quantise_row<XT, NORM>(static_cast<const XT*>(P.x), K, Kp, qs, redi, redd, P.gain,
+                                                   b.eps_norm, &sq, status, true);
+            if (tp == 0) {
+                s_scale[0] = s;
+                s_sumq[0] = sq;
             }
+        } else if constexpr (FUSED) {
+            // all rows at once; their loads go out ahead of the weight copies
+            named_bar_arrive(4, kThreads);
+            quantise_rows<MT, kConsumers, XT, NORM>(static_cast<const XT*>(P.x), M, K, P.gain, b.eps_norm, tp, qsh,
+                                                    ss_rows, s_scale, s_sumq, store_q, sync_consumers, status);
+            // words past K (the stores above stop at ceil(K/4))
+            const int kw0 = (K + 3) / 4;
+            for (int i = tp; i < M * (Kp / 4 - kw0); i += kConsumers)
+                store_q(i / (Kp / 4 - kw0), kw0 + i % (Kp / 4 - kw0), 0u);
         } else {
             named_bar_arrive(4, kThreads);
-#pragma unroll 1
-            for (int m = 0; m < M; ++m) {
-                const uint4* gq = reinterpret_cast<const uint4*>(P.q + (int64_t)m * Kp);
-                uint4* sq4 = reinterpret_cast<uint4*>(qs + m * Kp);
-                int part = 0;
-                for (int v = threadIdx.x - 32; v < Kp / 16; v += kConsumers) {
-                    const uint4 u = __ldg(gq + v);
-                    sq4[v] = u;
-                    part = dp4a_ss(u.x, 0x01010101u, part);
-                    part = dp4a_ss(u.y, 0x01010101u, part);
-                    part = dp4a_ss(u.z, 0x01010101u, part);
-                    part = dp4a_ss(u.w, 0x01010101u, part);
-                }
-                const int sq = consumers_sum(part, redi);
-                if (threadIdx.x == 32) {
-                    s_scale[m] = P.s[m];
-                    s_sumq[m] = sq;
-                }
-                named_bar(1, kConsumers);
-            }
+            copy_q_rows<MT, kConsumers>(P.q, M, Kp, tp, qsh, s_sumq, store_q, sync_consumers);
+            if (tp < M) s_scale[tp] = P.s[tp];
         }
         // token slots M .. MT-1 get zero activations, so the dot loop needs
         // no token guard (their sums are never written out)
