@@ -346,7 +346,7 @@ def run_decode(torch, bl, args, lin, M, dev, stream, dist, l2):
     S = setup_problems(torch, bl, lin, M, dev, 3 * l2, torch.float32)
     copies, Ns, Ks = S["copies"], S["Ns"], S["Ks"]
     mode = args.mode
-    if mode == "grouped" and any(bl_fused_too_big(bl, M, K) for K in Ks):
+    if mode == "grouped" and not all(bl.bitlinear_forward_x_supported(M, K) for K in Ks):
         mode = "separate"
     qs = [torch.empty((M, bl.bitlinear_padded_k(K)), dtype=torch.int8, device=dev) for K in Ks]
     gains = [(1.0 + 0.25 * torch.randn(K, generator=torch.Generator().manual_seed(K))).to(dev) for K in Ks]
@@ -372,7 +372,14 @@ def run_decode(torch, bl, args, lin, M, dev, stream, dist, l2):
                                  S["ys"][c][j], None, stream)
         return 2 * len(lin)
 
-    launches = step(0)
+    try:
+        launches = step(0)
+    except bl.BitLinearError as e:
+        # a forced decode kernel that cannot take the grouped fused form
+        if mode != "grouped" or e.status != bl.BL_ERR_SHAPE:
+            raise
+        mode = "separate"
+        launches = step(0)
     torch.cuda.synchronize()
     G = Graphs(torch, stream, step, copies)
     G.run(max(3, args.warmup))
@@ -406,11 +413,6 @@ def run_decode(torch, bl, args, lin, M, dev, stream, dist, l2):
         kname = f"{decode_kernel_name(args, M)} (product, one launch per linear)"
     return dict(S=S, mode=mode, ms=ms, launches=launches, clocks=clocks, nbytes=nbytes,
                 kern_ms=kern_ms, kern_bytes=kern_bytes, kname=kname)
-
-
-def bl_fused_too_big(bl, M, K):
-    p2 = 1 if M <= 1 else 2 if M <= 2 else 4 if M <= 4 else 8 if M <= 8 else 16
-    return M > 16 or p2 * bl.bitlinear_padded_k(K) > 160 * 1024
 
 
 def run_e2e(torch, bl, lin, M, dev, stream, S, steps, dist):

@@ -172,13 +172,25 @@ bl_status bitlinear_forward(const int8_t* q, const float* s, const uint8_t* pack
  * fused into the product kernel's prologue: x goes in, y comes out, q and s
  * never reach memory.  Results are identical to bitlinear_quant_act followed
  * by bitlinear_forward.  Arguments as in those two calls.
- * Errors: NULL, SHAPE (M, N, K <= 0; M > 16, or M' * Kp > 160 KiB with M'
- * = M rounded up to a power of two, for this fused decode form), ALIGN,
- * DTYPE, OVERFLOW, CUDA.
+ * Limits of this fused decode form: M <= 16, and the quantised activations
+ * of every problem must fit one CTA's shared memory: M' * Kp <= 160 KiB
+ * (M' = M rounded up to a power of two; every decode kernel), or else
+ * M' * Kp' <= 184 KiB with Kp' = Kp rounded up to a multiple of 4096 / M'
+ * (the tensor-core decode kernel only; e.g. M = 16 at K = 11008).
+ * Errors: NULL, SHAPE (M, N, K <= 0; the limits above; no kernel that the
+ * decode-kernel setting allows fits the shapes), ALIGN, DTYPE, OVERFLOW,
+ * CUDA.
  * ---------------------------------------------------------------------- */
 bl_status bitlinear_forward_x(const void* x, bl_dtype xt, const uint8_t* packed,
                               const float* gamma32, int64_t M, int64_t N, int64_t K, void* y,
                               bl_dtype yt, void* stream);
+
+/* Host-side query, no device work: 1 if the fused decode forms
+ * (bitlinear_forward_x, _grouped, _rmsnorm_grouped) accept M tokens of K
+ * columns under the limits above with BL_DECODE_AUTO, else 0 (also for M,
+ * K out of range).  Lets a caller choose between the fused form and
+ * bitlinear_quant_act + bitlinear_forward without trying. */
+int bitlinear_forward_x_supported(int64_t M, int64_t K);
 
 /* ------------------------------------------------------------------------
  * SubLN before the activation quantiser.  aratech.ae, "BitLinear: the
@@ -199,8 +211,8 @@ bl_status bitlinear_forward_x(const void* x, bl_dtype xt, const uint8_t* packed,
  *   bitlinear_forward_x_grouped with the normalisation in the prologue; each
  *   problem i has its own x[i] and gain[i] (pass the same pointers for
  *   linears that share one normalised input).  Same limits as that call
- *   (M <= 16, M' * Kp <= 160 KiB); BL_ERR_SHAPE also when neither streaming
- *   decode kernel fits, or when the per-tile kernel is forced (it has no
+ *   (bitlinear_forward_x); BL_ERR_SHAPE also when neither streaming decode
+ *   kernel fits, or when the per-tile kernel is forced (it has no
  *   normalising prologue).
  * ---------------------------------------------------------------------- */
 bl_status bitlinear_rmsnorm_quant_act(const void* x, bl_dtype xt, const float* gain, double eps, int64_t M,

@@ -34,6 +34,7 @@ SIGNATURES = {
     "bitlinear_forward": (_i32, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _i32, _vp, _vp]),
     "bitlinear_forward_x": (_i32, [_vp, _i32, _vp, _vp, _i64, _i64, _i64, _vp, _i32, _vp]),
     "bitlinear_forward_x_grouped": (_i32, [_i32, _vp, _i32, _vp, _vp, _i64, _vp, _vp, _vp, _i32, _vp]),
+    "bitlinear_forward_x_supported": (_i32, [_i64, _i64]),
     "bitlinear_rmsnorm_quant_act": (_i32, [_vp, _i32, _vp, C.c_double, _i64, _i64, _vp, _vp, _vp]),
     "bitlinear_forward_x_rmsnorm_grouped": (_i32, [_i32, _vp, _i32, _vp, C.c_double, _vp, _vp, _i64, _vp, _vp,
                                                    _vp, _i32, _vp]),
@@ -113,6 +114,11 @@ def _dtype_code(dt) -> int:
 # ------------------------------------------------------- C ABI mirror ----
 def bitlinear_padded_k(K: int) -> int:
     return int(lib().bitlinear_padded_k(K))
+
+
+def bitlinear_forward_x_supported(M: int, K: int) -> bool:
+    """Whether the fused decode forms take M tokens of K columns."""
+    return bool(lib().bitlinear_forward_x_supported(M, K))
 
 
 def bitlinear_packed_bytes(N: int, K: int) -> int:

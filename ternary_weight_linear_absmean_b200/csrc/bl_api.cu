@@ -218,13 +218,17 @@ bl_status bitlinear_forward_x_grouped(int count, const void* const* x, bl_dtype 
     b.count = count;
     b.M = M;
     int64_t tiles = 0;
+    bool tile_fits = true;   // the per-tile kernel holds M' * Kp of activations in shared memory
     for (int i = 0; i < count; ++i) {
         if (!x[i] || !packed[i] || !gamma32[i] || !y[i]) return BL_ERR_NULL;
         bl_status st = check_forward_shape(M, N[i], K[i]);
         if (st != BL_OK) return st;
-        if ((size_t)pow2_tokens(M) * (size_t)bl::padded_k(K[i]) > kFusedSmemLimit) return BL_ERR_SHAPE;
         if (!aligned16(x[i]) || !aligned16(packed[i]) || !aligned_to(gamma32[i], 4) || !aligned16(y[i]))
             return BL_ERR_ALIGN;
+        if ((size_t)pow2_tokens(M) * (size_t)bl::padded_k(K[i]) > kFusedSmemLimit) {
+            if (!bl::dec_tc_fits(M, K[i])) return BL_ERR_SHAPE;   // no decode kernel holds its activations
+            tile_fits = false;
+        }
         tiles += bl::padded_n(N[i]) / 8;
         b.p[i].x = x[i];
         b.p[i].packed = packed[i];
@@ -251,6 +255,7 @@ bl_status bitlinear_forward_x_grouped(int count, const void* const* x, bl_dtype 
     }
     const bl_status r = dispatch_decode(sb, true, xt, yt, status, cs);
     if (r != kTryNext) return r;
+    if (!tile_fits) return BL_ERR_SHAPE;
     return bl::launch_gemv(b, true, xt, yt, status, cs) == cudaSuccess ? BL_OK : BL_ERR_CUDA;
 }
 
@@ -283,7 +288,8 @@ bl_status bitlinear_forward_x_rmsnorm_grouped(int count, const void* const* x, b
         if (!x[i] || !gain[i] || !packed[i] || !gamma32[i] || !y[i]) return BL_ERR_NULL;
         bl_status st = check_forward_shape(M, N[i], K[i]);
         if (st != BL_OK) return st;
-        if ((size_t)pow2_tokens(M) * (size_t)bl::padded_k(K[i]) > kFusedSmemLimit) return BL_ERR_SHAPE;
+        if ((size_t)pow2_tokens(M) * (size_t)bl::padded_k(K[i]) > kFusedSmemLimit && !bl::dec_tc_fits(M, K[i]))
+            return BL_ERR_SHAPE;
         if (!aligned16(x[i]) || !aligned16(gain[i]) || !aligned16(packed[i]) || !aligned_to(gamma32[i], 4) ||
             !aligned16(y[i]))
             return BL_ERR_ALIGN;
@@ -308,6 +314,12 @@ bl_status bitlinear_forward_x(const void* x, bl_dtype xt, const uint8_t* packed,
                               int64_t M, int64_t N, int64_t K, void* y, bl_dtype yt, void* stream)
 {
     return bitlinear_forward_x_grouped(1, &x, xt, &packed, &gamma32, M, &N, &K, &y, yt, stream);
+}
+
+int bitlinear_forward_x_supported(int64_t M, int64_t K)
+{
+    if (check_forward_shape(M, 1, K) != BL_OK || M > bl::kFusedMaxM) return 0;
+    return ((size_t)pow2_tokens(M) * (size_t)bl::padded_k(K) <= kFusedSmemLimit || bl::dec_tc_fits(M, K)) ? 1 : 0;
 }
 
 bl_status bitlinear_get_status(void* stream)

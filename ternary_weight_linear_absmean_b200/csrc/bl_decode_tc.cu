@@ -82,7 +82,7 @@ constexpr uint32_t kIdescDec = idesc_i8(128, 16);
 constexpr int kPrefetch = 6;                 // stages in flight per expansion group (at most;
                                              // 4 or 2 when the resident operand is large)
 constexpr int kSmemBudget = 227 * 1024;     // static + dynamic, per CTA
-constexpr int kStaticReserve = 10 * 1024;   // barriers, ep[] (8 KiB at MT = 16), scratch
+constexpr int kStaticReserve = 10 * 1024;   // barriers, ep[] (4 KiB at MT = 8), scratch
 
 // Offset of the int8x4 activation word (k = 4*kw .. 4*kw+3, token m) in the
 // resident B operand.  The word's k fixes its chunk c = kw/16, the word
@@ -142,8 +142,6 @@ __global__ void __launch_bounds__(kThreads, 1) dec_tc_kernel(const __grid_consta
     // expansion groups' rings of D prefetched stages each
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* bres = base;
-    uint8_t* ring = base + b.q_bytes;
-    const int D = b.stages;                        // 2, 4 or 6
 
     // ---- problem and tile range of this CTA
     int pi = 0;
@@ -163,6 +161,14 @@ __global__ void __launch_bounds__(kThreads, 1) dec_tc_kernel(const __grid_consta
     const int J = job_stages<MT>(P.K);
     const int total = njobs * J;
     const uint32_t bres_bytes = (uint32_t)J * 2 * kAtom;
+    // The region was planned for the group's largest operand with rings of
+    // b.stages; a CTA of a problem with a smaller operand (shorter K) gives
+    // the difference to deeper rings: D = 2, 4 or 6 stages per group.
+    uint8_t* ring = base + bres_bytes;
+    const int D = [&] {
+        const uint32_t fit = ((uint32_t)b.q_bytes + 2u * (uint32_t)b.stages * kStage - bres_bytes) / (2u * kStage);
+        return fit >= (uint32_t)kPrefetch ? kPrefetch : fit >= 4 ? 4 : 2;
+    }();
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -482,6 +488,15 @@ int job_stages_rt(int MT, int64_t K)
 // operand (MT * Kp bytes, rounded up to whole stages) and two rings of 6
 // (else 4 or 2) 8 KiB stages.  MT (the operand's token slots, >= M) is the
 // largest for which that fits.
+// Whether one problem of M tokens and K columns fits the kernel's shared
+// memory at all: the resident operand of M's own slot count beside rings of
+// two stages.
+bool dec_tc_fits(int64_t M, int64_t K)
+{
+    const int64_t budget = kSmemBudget - kStaticReserve - 1024;
+    return M >= 1 && M <= 16 && (int64_t)job_stages_rt(stream_tokens(M), K) * 2 * kAtom + 2 * 2 * kStage <= budget;
+}
+
 bool plan_dec_tc(StreamBatch& b, int* grid, size_t* smem)
 {
     const int target = sm_count();

@@ -113,6 +113,7 @@ cudaError_t launch_stream(StreamBatch& b, bool fused, bl_dtype xt, bl_dtype yt, 
 // streaming kernel (plan fields are filled by its own planner).  Returns
 // cudaErrorNotSupported if the shapes do not fit (shared memory).
 bool plan_dec_tc(StreamBatch& b, int* grid, size_t* smem);
+bool dec_tc_fits(int64_t M, int64_t K);
 cudaError_t launch_dec_tc(StreamBatch& b, bool fused, bl_dtype xt, bl_dtype yt, unsigned* status,
                           cudaStream_t st);
 

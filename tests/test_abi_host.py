@@ -86,10 +86,29 @@ def test_forward_rejects_bad_arguments(L):
     assert (2 ** 31) // 127 == 16_909_320
 
 
+def test_forward_x_supported_query(L):
+    # host-side query of the fused forms' limits: M' * Kp <= 160 KiB (every
+    # decode kernel) or M' * Kp' <= 184 KiB with Kp' = Kp rounded up to a
+    # multiple of 4096 / M' (tensor-core kernel)
+    f = L.bitlinear_forward_x_supported
+    assert f(1, 2560) == 1
+    assert f(16, 10240) == 1                  # 160 KiB exactly
+    assert f(16, 11008) == 1                  # 172 KiB: tensor-core kernel only
+    assert f(16, 11776) == 1                  # 184 KiB exactly
+    assert f(16, 11777) == 0
+    assert f(9, 11776) == 1 and f(9, 12032) == 0   # M' = 16
+    assert f(8, 23552) == 1 and f(8, 23553) == 0   # Kp' multiple of 512
+    assert f(1, 188416) == 1 and f(1, 188417) == 0
+    assert f(17, 64) == 0 and f(0, 64) == 0 and f(1, 0) == 0
+
+
 def test_forward_x_rejects_bad_arguments(L):
     f = L.bitlinear_forward_x
     assert f(A, bl.BL_BF16, A, A, 17, 8, 64, A, bl.BL_F32, None) == bl.BL_ERR_SHAPE   # M > 16
-    assert f(A, bl.BL_BF16, A, A, 16, 8, 11008, A, bl.BL_F32, None) == bl.BL_ERR_SHAPE  # smem
+    # activations beyond every decode kernel's shared memory (16 x 12032 B;
+    # 16 x 11008 B still fits the tensor-core kernel)
+    assert f(A, bl.BL_BF16, A, A, 16, 8, 12032, A, bl.BL_F32, None) == bl.BL_ERR_SHAPE
+    assert f(A, bl.BL_BF16, A, A, 8, 8, 24000, A, bl.BL_F32, None) == bl.BL_ERR_SHAPE
     assert f(A, 5, A, A, 1, 8, 64, A, bl.BL_F32, None) == bl.BL_ERR_DTYPE
     assert f(MIS, bl.BL_BF16, A, A, 1, 8, 64, A, bl.BL_F32, None) == bl.BL_ERR_ALIGN
     g = L.bitlinear_forward_x_grouped

@@ -207,3 +207,49 @@ def test_prepared_grouped_call_matches_direct_call(bl):
     torch.cuda.synchronize()
     for a, b in zip(y1, y2):
         assert np.array_equal(a.cpu().numpy(), b.cpu().numpy())
+
+
+@pytest.mark.parametrize("M,N,K", [(16, 200, 11008), (12, 96, 11776), (1, 64, 150000)])
+def test_fused_beyond_the_streaming_limit(bl, M, N, K):
+    # activations above 160 KiB per CTA: only the tensor-core kernel holds
+    # them, and AUTO falls through to it for the fused form too
+    import torch
+    assert bl.bitlinear_forward_x_supported(M, K)
+    W = synth.weights(N, K, seed=K + 5 * M)
+    x = synth.activations(M, K, seed=M + K, dtype="bf16", outlier_frac=0.01)
+    ref = oracle.bitlinear(W, x, "bf16")
+    packed, _, g32 = _packed(bl, W)
+    y = bl.forward_x(P.to_dev_bf16(x), packed, g32, N, K)
+    torch.cuda.synchronize()
+    assert bl.bitlinear_get_status() == bl.BL_OK
+    P.check_y_f32(y.cpu().numpy(), ref["y"], exact=True)
+    bl.bitlinear_set_decode_kernel(bl.BL_DECODE_DP4A)
+    try:
+        with pytest.raises(bl.BitLinearError):
+            bl.forward_x(P.to_dev_bf16(x), packed, g32, N, K)
+    finally:
+        bl.bitlinear_set_decode_kernel(bl.BL_DECODE_AUTO)
+
+
+@pytest.mark.parametrize("M", [9, 16])
+def test_grouped_mixed_ring_depths(bl, M):
+    # one launch over a long-K problem (shallow rings) and short-K problems
+    # (their CTAs take deeper rings from the same shared-memory region)
+    import torch
+    shapes = [(96, 11008), (200, 4096), (64, 1000), (8, 64)]
+    xs, ps, gs, ys, refs = [], [], [], [], []
+    for i, (N, K) in enumerate(shapes):
+        W = synth.weights(N, K, seed=700 + i)
+        x = synth.activations(M, K, seed=800 + i, dtype="bf16", outlier_frac=0.01)
+        refs.append(oracle.bitlinear(W, x, "bf16"))
+        p, _, g = _packed(bl, W)
+        xs.append(P.to_dev_bf16(x))
+        ps.append(p)
+        gs.append(g)
+        ys.append(torch.empty((M, N), dtype=torch.float32, device="cuda"))
+    bl.bitlinear_forward_x_grouped(xs, ps, gs, [s[0] for s in shapes], [s[1] for s in shapes], ys)
+    torch.cuda.synchronize()
+    assert bl.bitlinear_get_status() == bl.BL_OK
+    for y, ref in zip(ys, refs):
+        P.check_y_f32(y.cpu().numpy(), ref["y"], exact=True)
+

@@ -136,3 +136,29 @@ def test_rmsnorm_then_prefill_gemm(bl):
     assert straddle_rows(x, "bf16", eps).sum() == 0
     assert np.array_equal(acc.cpu().numpy(), ref["acc"])
     P.check_y_f32(y.cpu().numpy(), ref["y"])
+
+
+def test_rmsnorm_grouped_beyond_the_streaming_limit(bl):
+    # M = 16 at K = 11008: the activations fit only the tensor-core kernel
+    import torch
+    M, eps, shapes = 16, 1e-6, [(64, 11008), (128, 4096)]
+    xs, gains, ps, gs, ys, refs, xs_host = [], [], [], [], [], [], []
+    for i, (N, K) in enumerate(shapes):
+        W = synth.weights(N, K, seed=900 + i)
+        x = synth.activations(M, K, seed=910 + i, dtype="bf16", outlier_frac=0.01)
+        g = _gain(K, 920 + i)
+        refs.append(oracle.bitlinear_rmsnorm(W, x, "bf16", g, eps))
+        p, _, g32 = bl.pack(P.to_dev_f32(W))
+        xs.append(P.to_dev_bf16(x))
+        xs_host.append(x)
+        gains.append(P.to_dev_f32(g))
+        ps.append(p)
+        gs.append(g32)
+        ys.append(torch.empty((M, N), dtype=torch.float32, device="cuda"))
+    bl.bitlinear_forward_x_rmsnorm_grouped(xs, gains, eps, ps, gs, [s[0] for s in shapes],
+                                           [s[1] for s in shapes], ys)
+    torch.cuda.synchronize()
+    assert bl.bitlinear_get_status() == bl.BL_OK
+    assert all(straddle_rows(x, "bf16", eps).sum() == 0 for x in xs_host)
+    for y, ref in zip(ys, refs):
+        P.check_y_f32(y.cpu().numpy(), ref["y"], exact=True)
