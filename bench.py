@@ -352,15 +352,21 @@ def run_decode(torch, bl, args, lin, M, dev, stream, dist, l2):
     gains = [(1.0 + 0.25 * torch.randn(K, generator=torch.Generator().manual_seed(K))).to(dev) for K in Ks]
     ss = [torch.empty(M, dtype=torch.float32, device=dev) for _ in Ks]
 
+    # the workspace form: for M >= 2 one quantiser launch over all linears,
+    # then the product kernel on the codes
+    ws = bl.decode_workspace(M, Ks, dev) if mode == "grouped" else None
+    grouped_launches = 2 if M >= 2 else 1
+
     def step(i):
         c = i % copies
         if mode == "grouped" and args.rmsnorm:
             bl.bitlinear_forward_x_rmsnorm_grouped(S["xs"][c], gains, 1e-6, S["packed"][c], S["g32"], Ns, Ks,
-                                                   S["ys"][c], stream)
-            return 1
+                                                   S["ys"][c], stream, workspace=ws)
+            return grouped_launches
         if mode == "grouped":
-            bl.bitlinear_forward_x_grouped(S["xs"][c], S["packed"][c], S["g32"], Ns, Ks, S["ys"][c], stream)
-            return 1
+            bl.bitlinear_forward_x_grouped(S["xs"][c], S["packed"][c], S["g32"], Ns, Ks, S["ys"][c], stream,
+                                           workspace=ws)
+            return grouped_launches
         if mode == "fused":
             for j in range(len(lin)):
                 bl.bitlinear_forward_x(S["xs"][c][j], S["packed"][c][j], S["g32"][j], Ns[j], Ks[j],
@@ -392,8 +398,12 @@ def run_decode(torch, bl, args, lin, M, dev, stream, dist, l2):
     nbytes = decode_bytes(lin, M)
 
     # dominant kernel: the product kernel (the whole step in grouped mode)
-    if mode == "grouped":
+    if mode == "grouped" and M == 1:
         kern_ms, kern_bytes, kname = ms / args.steps, nbytes, f"{decode_kernel_name(args, M)} (fused quantise, {len(lin)} linears, 1 launch)"
+    elif mode == "grouped":
+        # the whole step (quantiser + product kernel) against the product's
+        # bytes: a lower bound on the product kernel's own rate
+        kern_ms, kern_bytes, kname = ms / args.steps, nbytes, f"quant_kernel + {decode_kernel_name(args, M)} (product on the codes, {len(lin)} linears, 2 launches; both timed)"
     else:
         def kstep(i):
             c = i % copies

@@ -263,6 +263,38 @@ bl_status bitlinear_forward_x_grouped(int count, const void* const* x, bl_dtype 
                                       int64_t M, const int64_t* N, const int64_t* K,
                                       void* const* y, bl_dtype yt, void* stream);
 
+/* ------------------------------------------------------------------------
+ * Workspace forms of the grouped fused decode calls.  Same arguments,
+ * results (bit for bit) and errors as bitlinear_forward_x_grouped and
+ * bitlinear_forward_x_rmsnorm_grouped, plus a device workspace (16-byte
+ * aligned, caller-owned, at least bitlinear_decode_workspace_bytes(count,
+ * M, K) bytes, else BL_ERR_WORKSPACE; NULL: BL_ERR_NULL) that the call may
+ * overwrite, in stream order.  For M >= 2 the call quantises every token
+ * row once, in a launch of its own (bitlinear_quant_act's kernel, over all
+ * problems), into the workspace and then runs the product kernel on the
+ * codes: in the single-launch form each CTA of the product kernel
+ * quantises all M rows of its problem itself, reading x from L2 twice, which
+ * costs more than a second launch once M > 1.  For M = 1 the workspace is
+ * not touched and the call is the single-launch form.  Two calls in flight
+ * at once (different streams) need different workspaces.
+ *
+ * bitlinear_decode_workspace_bytes -- the bytes those calls need: per
+ * problem M * Kp bytes of codes and M fp32 scales, each rounded up to 256.
+ * Host-only; 0 for count outside 1..16, K NULL, M outside 1..16 or a K
+ * outside 1..16,909,320.
+ * ---------------------------------------------------------------------- */
+int64_t bitlinear_decode_workspace_bytes(int count, int64_t M, const int64_t* K);
+bl_status bitlinear_forward_x_grouped_ws(int count, const void* const* x, bl_dtype xt,
+                                         const uint8_t* const* packed, const float* const* gamma32, int64_t M,
+                                         const int64_t* N, const int64_t* K, void* const* y, bl_dtype yt,
+                                         void* workspace, int64_t workspace_bytes, void* stream);
+bl_status bitlinear_forward_x_rmsnorm_grouped_ws(int count, const void* const* x, bl_dtype xt,
+                                                 const float* const* gain, double eps,
+                                                 const uint8_t* const* packed, const float* const* gamma32,
+                                                 int64_t M, const int64_t* N, const int64_t* K, void* const* y,
+                                                 bl_dtype yt, void* workspace, int64_t workspace_bytes,
+                                                 void* stream);
+
 /* Synchronises `stream`, then returns and clears the device status word of
  * the current device: BL_OK; BL_ERR_TIMEOUT if a kernel abandoned one of its
  * bounded waits (its outputs are then invalid); else BL_ERR_NONFINITE if a

@@ -35,6 +35,11 @@ SIGNATURES = {
     "bitlinear_forward_x": (_i32, [_vp, _i32, _vp, _vp, _i64, _i64, _i64, _vp, _i32, _vp]),
     "bitlinear_forward_x_grouped": (_i32, [_i32, _vp, _i32, _vp, _vp, _i64, _vp, _vp, _vp, _i32, _vp]),
     "bitlinear_forward_x_supported": (_i32, [_i64, _i64]),
+    "bitlinear_decode_workspace_bytes": (_i64, [_i32, _i64, _vp]),
+    "bitlinear_forward_x_grouped_ws": (_i32, [_i32, _vp, _i32, _vp, _vp, _i64, _vp, _vp, _vp, _i32, _vp, _i64,
+                                              _vp]),
+    "bitlinear_forward_x_rmsnorm_grouped_ws": (_i32, [_i32, _vp, _i32, _vp, C.c_double, _vp, _vp, _i64, _vp, _vp,
+                                                      _vp, _i32, _vp, _i64, _vp]),
     "bitlinear_rmsnorm_quant_act": (_i32, [_vp, _i32, _vp, C.c_double, _i64, _i64, _vp, _vp, _vp]),
     "bitlinear_forward_x_rmsnorm_grouped": (_i32, [_i32, _vp, _i32, _vp, C.c_double, _vp, _vp, _i64, _vp, _vp,
                                                    _vp, _i32, _vp]),
@@ -170,18 +175,42 @@ def bitlinear_forward_x(x, packed, gamma32, N, K, y, stream=None) -> None:
     _check(st, "bitlinear_forward_x")
 
 
-def bitlinear_forward_x_grouped(xs, packeds, gammas, Ns, Ks, ys, stream=None) -> None:
+def bitlinear_decode_workspace_bytes(M: int, Ks) -> int:
+    """Device workspace bytes of the grouped calls' workspace forms."""
+    n = len(Ks)
+    return int(lib().bitlinear_decode_workspace_bytes(n, M, (C.c_int64 * n)(*Ks)))
+
+
+def decode_workspace(M: int, Ks, device):
+    """A workspace tensor for the grouped calls (uint8, device)."""
+    torch = _torch()
+    nbytes = bitlinear_decode_workspace_bytes(M, Ks)
+    if nbytes <= 0:
+        raise ValueError("no workspace size for these shapes")
+    return torch.empty(nbytes, dtype=torch.uint8, device=device)
+
+
+def _ws_args(workspace):
+    return _dptr(workspace, "workspace"), workspace.numel() * workspace.element_size()
+
+
+def bitlinear_forward_x_grouped(xs, packeds, gammas, Ns, Ks, ys, stream=None, workspace=None) -> None:
+    """One launch over the problems; with a workspace (decode_workspace)
+    and M >= 2, a quantiser launch first and the product on the codes."""
     n = len(xs)
     if not (len(packeds) == len(gammas) == len(Ns) == len(Ks) == len(ys) == n):
         raise ValueError("grouped arguments must all have the same length")
     M = xs[0].shape[0]
     arr_p = C.c_void_p * n
     arr_i = C.c_int64 * n
-    st = lib().bitlinear_forward_x_grouped(
-        n, arr_p(*[_dptr(t, "x") for t in xs]), _dtype_code(xs[0].dtype),
-        arr_p(*[_dptr(t, "packed") for t in packeds]), arr_p(*[_dptr(t, "gamma32") for t in gammas]), M,
-        arr_i(*Ns), arr_i(*Ks), arr_p(*[_dptr(t, "y") for t in ys]), _dtype_code(ys[0].dtype), _stream(stream))
-    _check(st, "bitlinear_forward_x_grouped")
+    args = (n, arr_p(*[_dptr(t, "x") for t in xs]), _dtype_code(xs[0].dtype),
+            arr_p(*[_dptr(t, "packed") for t in packeds]), arr_p(*[_dptr(t, "gamma32") for t in gammas]), M,
+            arr_i(*Ns), arr_i(*Ks), arr_p(*[_dptr(t, "y") for t in ys]), _dtype_code(ys[0].dtype))
+    if workspace is None:
+        _check(lib().bitlinear_forward_x_grouped(*args, _stream(stream)), "bitlinear_forward_x_grouped")
+    else:
+        _check(lib().bitlinear_forward_x_grouped_ws(*args, *_ws_args(workspace), _stream(stream)),
+               "bitlinear_forward_x_grouped_ws")
 
 
 def bitlinear_rmsnorm_quant_act(x, gain, eps, q, s, stream=None) -> None:
@@ -191,41 +220,56 @@ def bitlinear_rmsnorm_quant_act(x, gain, eps, q, s, stream=None) -> None:
     _check(st, "bitlinear_rmsnorm_quant_act")
 
 
-def bitlinear_forward_x_rmsnorm_grouped(xs, gains, eps, packeds, gammas, Ns, Ks, ys, stream=None) -> None:
+def bitlinear_forward_x_rmsnorm_grouped(xs, gains, eps, packeds, gammas, Ns, Ks, ys, stream=None,
+                                        workspace=None) -> None:
     n = len(xs)
     if not (len(gains) == len(packeds) == len(gammas) == len(Ns) == len(Ks) == len(ys) == n):
         raise ValueError("grouped arguments must all have the same length")
     M = xs[0].shape[0]
     arr_p = C.c_void_p * n
     arr_i = C.c_int64 * n
-    st = lib().bitlinear_forward_x_rmsnorm_grouped(
-        n, arr_p(*[_dptr(t, "x") for t in xs]), _dtype_code(xs[0].dtype), arr_p(*[_dptr(t, "gain") for t in gains]),
-        float(eps), arr_p(*[_dptr(t, "packed") for t in packeds]), arr_p(*[_dptr(t, "gamma32") for t in gammas]),
-        M, arr_i(*Ns), arr_i(*Ks), arr_p(*[_dptr(t, "y") for t in ys]), _dtype_code(ys[0].dtype), _stream(stream))
-    _check(st, "bitlinear_forward_x_rmsnorm_grouped")
+    args = (n, arr_p(*[_dptr(t, "x") for t in xs]), _dtype_code(xs[0].dtype), arr_p(*[_dptr(t, "gain") for t in gains]),
+            float(eps), arr_p(*[_dptr(t, "packed") for t in packeds]), arr_p(*[_dptr(t, "gamma32") for t in gammas]),
+            M, arr_i(*Ns), arr_i(*Ks), arr_p(*[_dptr(t, "y") for t in ys]), _dtype_code(ys[0].dtype))
+    if workspace is None:
+        _check(lib().bitlinear_forward_x_rmsnorm_grouped(*args, _stream(stream)),
+               "bitlinear_forward_x_rmsnorm_grouped")
+    else:
+        _check(lib().bitlinear_forward_x_rmsnorm_grouped_ws(*args, *_ws_args(workspace), _stream(stream)),
+               "bitlinear_forward_x_rmsnorm_grouped_ws")
 
 
 class GroupedDecode:
-    """A prepared bitlinear_forward_x_grouped call: the pointer and size
-    arrays are marshalled once, so each call costs one C call (for decode
-    loops that run the same layers every token).  The tensors must stay
-    alive and in place while the object is used."""
+    """A prepared grouped decode call (bitlinear_forward_x_grouped_ws, or
+    its SubLN form when gains are given): the pointer and size arrays are
+    marshalled and the workspace allocated once, so each call costs one C
+    call (for decode loops that run the same layers every token).  The
+    tensors must stay alive and in place while the object is used, and one
+    object must not run on two streams at once (they share the workspace)."""
 
-    def __init__(self, xs, packeds, gammas, Ns, Ks, ys):
+    def __init__(self, xs, packeds, gammas, Ns, Ks, ys, gains=None, eps=1e-6):
         n = len(xs)
         if not (len(packeds) == len(gammas) == len(Ns) == len(Ks) == len(ys) == n):
             raise ValueError("grouped arguments must all have the same length")
+        if gains is not None and len(gains) != n:
+            raise ValueError("grouped arguments must all have the same length")
         arr_p = C.c_void_p * n
         arr_i = C.c_int64 * n
-        self._keep = (list(xs), list(packeds), list(gammas), list(ys))
-        self._args = (n, arr_p(*[_dptr(t, "x") for t in xs]), _dtype_code(xs[0].dtype),
-                      arr_p(*[_dptr(t, "packed") for t in packeds]), arr_p(*[_dptr(t, "gamma32") for t in gammas]),
-                      xs[0].shape[0], arr_i(*Ns), arr_i(*Ks), arr_p(*[_dptr(t, "y") for t in ys]),
-                      _dtype_code(ys[0].dtype))
-        self._fn = lib().bitlinear_forward_x_grouped
+        M = xs[0].shape[0]
+        self.workspace = decode_workspace(M, Ks, xs[0].device)
+        self._keep = (list(xs), list(packeds), list(gammas), list(ys), list(gains or []))
+        head = (n, arr_p(*[_dptr(t, "x") for t in xs]), _dtype_code(xs[0].dtype))
+        if gains is not None:
+            head += (arr_p(*[_dptr(t, "gain") for t in gains]), float(eps))
+        self._args = head + (arr_p(*[_dptr(t, "packed") for t in packeds]),
+                             arr_p(*[_dptr(t, "gamma32") for t in gammas]), M, arr_i(*Ns), arr_i(*Ks),
+                             arr_p(*[_dptr(t, "y") for t in ys]), _dtype_code(ys[0].dtype),
+                             *_ws_args(self.workspace))
+        self._name = "bitlinear_forward_x_rmsnorm_grouped_ws" if gains is not None else "bitlinear_forward_x_grouped_ws"
+        self._fn = getattr(lib(), self._name)
 
     def __call__(self, stream=None) -> None:
-        _check(self._fn(*self._args, _stream(stream)), "bitlinear_forward_x_grouped")
+        _check(self._fn(*self._args, _stream(stream)), self._name)
 
 
 def bitlinear_get_status(stream=None) -> int:

@@ -71,6 +71,137 @@ bl_status check_forward_shape(int64_t M, int64_t N, int64_t K)
     return BL_OK;
 }
 
+// Workspace of the calls that quantise in a launch of their own: per
+// problem its int8 codes [M][Kp], then its fp32 scales [M], each at a
+// 256-byte aligned offset.  Returns the total; fills the pointers if given.
+int64_t ws_layout(int count, int64_t M, const int64_t* K, void* ws, int8_t** q, float** s)
+{
+    auto up = [](int64_t v) { return (v + 255) / 256 * 256; };
+    int64_t off = 0;
+    for (int i = 0; i < count; ++i) {
+        if (q) q[i] = reinterpret_cast<int8_t*>(static_cast<char*>(ws) + off);
+        off += up(M * bl::padded_k(K[i]));
+        if (s) s[i] = reinterpret_cast<float*>(static_cast<char*>(ws) + off);
+        off += up(4 * M);
+    }
+    return off;
+}
+
+// Token count from which the calls given a workspace quantise every row
+// once, in a launch of their own, and run the product kernel on the codes:
+// each CTA of a fused product kernel quantises all M rows itself, so the
+// CTAs together read x (M x K) twice each from L2, which costs more than a
+// second launch once M > 1.
+constexpr int64_t kSplitMinM = 2;
+
+// The grouped fused decode calls (bitlinear_forward_x_grouped and its
+// SubLN and workspace forms).  gain: NULL, or one gain vector per problem.
+bl_status grouped_decode(int count, const void* const* x, bl_dtype xt, const float* const* gain, double eps,
+                         const uint8_t* const* packed, const float* const* gamma32, int64_t M, const int64_t* N,
+                         const int64_t* K, void* const* y, bl_dtype yt, void* ws, int64_t ws_bytes, bool has_ws,
+                         void* stream)
+{
+    if (count < 1 || count > bl::kMaxGroup) return BL_ERR_ARG;
+    if (!x || !packed || !gamma32 || !N || !K || !y) return BL_ERR_NULL;
+    if (check_dtype(xt) != BL_OK || check_dtype(yt) != BL_OK) return BL_ERR_DTYPE;
+    if (M <= 0 || M > bl::kFusedMaxM) return BL_ERR_SHAPE;
+    if (gain && (!(eps >= 0.0) || !std::isfinite(eps))) return BL_ERR_ARG;
+    bl::GemvBatch b;
+    std::memset(&b, 0, sizeof(b));
+    b.count = count;
+    b.M = M;
+    int64_t tiles = 0;
+    bool tile_fits = true;   // the per-tile kernel holds M' * Kp of activations in shared memory
+    for (int i = 0; i < count; ++i) {
+        if (!x[i] || !packed[i] || !gamma32[i] || !y[i] || (gain && !gain[i])) return BL_ERR_NULL;
+        bl_status st = check_forward_shape(M, N[i], K[i]);
+        if (st != BL_OK) return st;
+        if ((size_t)pow2_tokens(M) * (size_t)bl::padded_k(K[i]) > kFusedSmemLimit) {
+            if (!bl::dec_tc_fits(M, K[i])) return BL_ERR_SHAPE;   // no decode kernel holds its activations
+            tile_fits = false;
+        }
+        if (!aligned16(x[i]) || !aligned16(packed[i]) || !aligned_to(gamma32[i], 4) || !aligned16(y[i]) ||
+            (gain && !aligned16(gain[i])))
+            return BL_ERR_ALIGN;
+        tiles += bl::padded_n(N[i]) / 8;
+        b.p[i].x = x[i];
+        b.p[i].packed = packed[i];
+        b.p[i].gamma32 = gamma32[i];
+        b.p[i].y = y[i];
+        b.p[i].N = N[i];
+        b.p[i].K = K[i];
+    }
+    if (tiles > (int64_t(1) << 31) - 1) return BL_ERR_SHAPE;
+    if (has_ws) {
+        if (!ws) return BL_ERR_NULL;
+        if (!aligned16(ws)) return BL_ERR_ALIGN;
+        if (ws_bytes < ws_layout(count, M, K, nullptr, nullptr, nullptr)) return BL_ERR_WORKSPACE;
+    }
+    unsigned* status = status_word();
+    if (!status) return BL_ERR_CUDA;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    bl::StreamBatch sb;
+    std::memset(&sb, 0, sizeof(sb));
+    sb.count = count;
+    sb.M = (int)M;
+    sb.eps_norm = eps;
+    for (int i = 0; i < count; ++i) {
+        sb.p[i].x = x[i];
+        sb.p[i].gain = gain ? gain[i] : nullptr;
+        sb.p[i].packed = packed[i];
+        sb.p[i].gamma32 = gamma32[i];
+        sb.p[i].y = y[i];
+        sb.p[i].N = N[i];
+        sb.p[i].K = K[i];
+    }
+    const int kind = g_decode_kernel.load();
+    if (has_ws && M >= kSplitMinM && kind != BL_DECODE_LUT) {
+        // every row quantised once (one launch), then the product on the codes
+        int8_t* q[bl::kMaxGroup];
+        float* s[bl::kMaxGroup];
+        ws_layout(count, M, K, ws, q, s);
+        bl::QuantBatch qb;
+        std::memset(&qb, 0, sizeof(qb));
+        qb.count = count;
+        qb.rows = (int)(M * count);
+        qb.eps = eps;
+        for (int i = 0; i < count; ++i) {
+            qb.p[i].x = x[i];
+            qb.p[i].gain = gain ? gain[i] : nullptr;
+            qb.p[i].q = q[i];
+            qb.p[i].s = s[i];
+            qb.p[i].K = K[i];
+            qb.p[i].row_begin = (int)(M * i);
+            qb.row_begin[i] = qb.p[i].row_begin;
+            sb.p[i].x = nullptr;
+            sb.p[i].gain = nullptr;
+            sb.p[i].q = q[i];
+            sb.p[i].s = s[i];
+            b.p[i].x = nullptr;
+            b.p[i].q = q[i];
+            b.p[i].s = s[i];
+        }
+        if (bl::launch_quant_grouped(qb, xt, status, cs) != cudaSuccess) return BL_ERR_CUDA;
+        const bl_status r = dispatch_decode(sb, false, BL_F32, yt, status, cs);
+        if (r != kTryNext) return r;
+        // the per-tile kernel's unfused form takes one problem per launch
+        for (int i = 0; i < count; ++i) {
+            bl::GemvBatch one;
+            std::memset(&one, 0, sizeof(one));
+            one.count = 1;
+            one.M = M;
+            one.p[0] = b.p[i];
+            if (bl::launch_gemv(one, false, BL_F32, yt, status, cs) != cudaSuccess) return BL_ERR_CUDA;
+        }
+        return BL_OK;
+    }
+    const bl_status r = dispatch_decode(sb, true, xt, yt, status, cs);
+    if (r != kTryNext) return r;
+    // the per-tile kernel has no normalising prologue
+    if (gain || !tile_fits) return BL_ERR_SHAPE;
+    return bl::launch_gemv(b, true, xt, yt, status, cs) == cudaSuccess ? BL_OK : BL_ERR_CUDA;
+}
+
 }  // namespace
 
 namespace bl {
@@ -209,54 +340,24 @@ bl_status bitlinear_forward_x_grouped(int count, const void* const* x, bl_dtype 
                                       int64_t M, const int64_t* N, const int64_t* K, void* const* y,
                                       bl_dtype yt, void* stream)
 {
-    if (count < 1 || count > bl::kMaxGroup) return BL_ERR_ARG;
-    if (!x || !packed || !gamma32 || !N || !K || !y) return BL_ERR_NULL;
-    if (check_dtype(xt) != BL_OK || check_dtype(yt) != BL_OK) return BL_ERR_DTYPE;
-    if (M <= 0 || M > bl::kFusedMaxM) return BL_ERR_SHAPE;
-    bl::GemvBatch b;
-    std::memset(&b, 0, sizeof(b));
-    b.count = count;
-    b.M = M;
-    int64_t tiles = 0;
-    bool tile_fits = true;   // the per-tile kernel holds M' * Kp of activations in shared memory
-    for (int i = 0; i < count; ++i) {
-        if (!x[i] || !packed[i] || !gamma32[i] || !y[i]) return BL_ERR_NULL;
-        bl_status st = check_forward_shape(M, N[i], K[i]);
-        if (st != BL_OK) return st;
-        if (!aligned16(x[i]) || !aligned16(packed[i]) || !aligned_to(gamma32[i], 4) || !aligned16(y[i]))
-            return BL_ERR_ALIGN;
-        if ((size_t)pow2_tokens(M) * (size_t)bl::padded_k(K[i]) > kFusedSmemLimit) {
-            if (!bl::dec_tc_fits(M, K[i])) return BL_ERR_SHAPE;   // no decode kernel holds its activations
-            tile_fits = false;
-        }
-        tiles += bl::padded_n(N[i]) / 8;
-        b.p[i].x = x[i];
-        b.p[i].packed = packed[i];
-        b.p[i].gamma32 = gamma32[i];
-        b.p[i].y = y[i];
-        b.p[i].N = N[i];
-        b.p[i].K = K[i];
-    }
-    if (tiles > (int64_t(1) << 31) - 1) return BL_ERR_SHAPE;
-    unsigned* status = status_word();
-    if (!status) return BL_ERR_CUDA;
-    cudaStream_t cs = static_cast<cudaStream_t>(stream);
-    bl::StreamBatch sb;
-    std::memset(&sb, 0, sizeof(sb));
-    sb.count = count;
-    sb.M = (int)M;
-    for (int i = 0; i < count; ++i) {
-        sb.p[i].x = x[i];
-        sb.p[i].packed = packed[i];
-        sb.p[i].gamma32 = gamma32[i];
-        sb.p[i].y = y[i];
-        sb.p[i].N = N[i];
-        sb.p[i].K = K[i];
-    }
-    const bl_status r = dispatch_decode(sb, true, xt, yt, status, cs);
-    if (r != kTryNext) return r;
-    if (!tile_fits) return BL_ERR_SHAPE;
-    return bl::launch_gemv(b, true, xt, yt, status, cs) == cudaSuccess ? BL_OK : BL_ERR_CUDA;
+    return grouped_decode(count, x, xt, nullptr, 0.0, packed, gamma32, M, N, K, y, yt, nullptr, 0, false, stream);
+}
+
+bl_status bitlinear_forward_x_grouped_ws(int count, const void* const* x, bl_dtype xt,
+                                         const uint8_t* const* packed, const float* const* gamma32, int64_t M,
+                                         const int64_t* N, const int64_t* K, void* const* y, bl_dtype yt,
+                                         void* workspace, int64_t workspace_bytes, void* stream)
+{
+    return grouped_decode(count, x, xt, nullptr, 0.0, packed, gamma32, M, N, K, y, yt, workspace,
+                          workspace_bytes, true, stream);
+}
+
+int64_t bitlinear_decode_workspace_bytes(int count, int64_t M, const int64_t* K)
+{
+    if (count < 1 || count > bl::kMaxGroup || !K || M <= 0 || M > bl::kFusedMaxM) return 0;
+    for (int i = 0; i < count; ++i)
+        if (K[i] <= 0 || K[i] > kMaxK) return 0;
+    return ws_layout(count, M, K, nullptr, nullptr, nullptr);
 }
 
 int bitlinear_set_decode_kernel(int kind)
@@ -273,41 +374,20 @@ bl_status bitlinear_forward_x_rmsnorm_grouped(int count, const void* const* x, b
                                               const float* const* gamma32, int64_t M, const int64_t* N,
                                               const int64_t* K, void* const* y, bl_dtype yt, void* stream)
 {
-    if (count < 1 || count > bl::kMaxGroup) return BL_ERR_ARG;
-    if (!x || !gain || !packed || !gamma32 || !N || !K || !y) return BL_ERR_NULL;
-    if (check_dtype(xt) != BL_OK || check_dtype(yt) != BL_OK) return BL_ERR_DTYPE;
-    if (M <= 0 || M > bl::kFusedMaxM) return BL_ERR_SHAPE;
-    if (!(eps >= 0.0) || !std::isfinite(eps)) return BL_ERR_ARG;
-    bl::StreamBatch sb;
-    std::memset(&sb, 0, sizeof(sb));
-    sb.count = count;
-    sb.M = (int)M;
-    sb.eps_norm = eps;
-    int64_t tiles = 0;
-    for (int i = 0; i < count; ++i) {
-        if (!x[i] || !gain[i] || !packed[i] || !gamma32[i] || !y[i]) return BL_ERR_NULL;
-        bl_status st = check_forward_shape(M, N[i], K[i]);
-        if (st != BL_OK) return st;
-        if ((size_t)pow2_tokens(M) * (size_t)bl::padded_k(K[i]) > kFusedSmemLimit && !bl::dec_tc_fits(M, K[i]))
-            return BL_ERR_SHAPE;
-        if (!aligned16(x[i]) || !aligned16(gain[i]) || !aligned16(packed[i]) || !aligned_to(gamma32[i], 4) ||
-            !aligned16(y[i]))
-            return BL_ERR_ALIGN;
-        tiles += bl::padded_n(N[i]) / 8;
-        sb.p[i].x = x[i];
-        sb.p[i].gain = gain[i];
-        sb.p[i].packed = packed[i];
-        sb.p[i].gamma32 = gamma32[i];
-        sb.p[i].y = y[i];
-        sb.p[i].N = N[i];
-        sb.p[i].K = K[i];
-    }
-    if (tiles > (int64_t(1) << 31) - 1) return BL_ERR_SHAPE;
-    unsigned* status = status_word();
-    if (!status) return BL_ERR_CUDA;
-    const bl_status r = dispatch_decode(sb, true, xt, yt, status, static_cast<cudaStream_t>(stream));
-    // the per-tile kernel has no normalising prologue
-    return r == kTryNext ? BL_ERR_SHAPE : r;
+    if (!gain) return BL_ERR_NULL;
+    return grouped_decode(count, x, xt, gain, eps, packed, gamma32, M, N, K, y, yt, nullptr, 0, false, stream);
+}
+
+bl_status bitlinear_forward_x_rmsnorm_grouped_ws(int count, const void* const* x, bl_dtype xt,
+                                                 const float* const* gain, double eps,
+                                                 const uint8_t* const* packed, const float* const* gamma32,
+                                                 int64_t M, const int64_t* N, const int64_t* K, void* const* y,
+                                                 bl_dtype yt, void* workspace, int64_t workspace_bytes,
+                                                 void* stream)
+{
+    if (!gain) return BL_ERR_NULL;
+    return grouped_decode(count, x, xt, gain, eps, packed, gamma32, M, N, K, y, yt, workspace, workspace_bytes,
+                          true, stream);
 }
 
 bl_status bitlinear_forward_x(const void* x, bl_dtype xt, const uint8_t* packed, const float* gamma32,

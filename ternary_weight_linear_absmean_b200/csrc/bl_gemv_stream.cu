@@ -102,7 +102,7 @@ __device__ __forceinline__ uint32_t pack4(int a, int b, int c, int d)
 // cleared -- for non-negative IEEE values integer order is numeric order,
 // and NaN/Inf patterns sort above every finite value, so the same max also
 // flags non-finite input; (2) rint + clamp + convert is one
-// round-to-nearest-even conversion, since |x * s| < 127.5 for finite x (the
+// round-to-nearest-even addition (rint_low_byte), since |x * s| < 127.5 for finite x (the
 // clamp can never bind).
 template <typename XT, bool NORM>
 __device__ float quantise_row(const XT* __restrict__ row, int K, int Kp, int8_t* q, int* redi, double* redd,
@@ -226,7 +226,7 @@ __device__ float quantise_row(const XT* __restrict__ row, int K, int Kp, int8_t*
                 for (int b = 0; b < 4; ++b) {
                     float e = elem(u, 4 * p + b);
                     if constexpr (NORM) e = __fmul_rn(__fmul_rn(e, r32), g[4 * p + b]);
-                    c[b] = __float2int_rn(__fmul_rn(e, s));
+                    c[b] = (int)rint_low_byte(__fmul_rn(e, s));
                 }
                 w[p] = pack4(c[0], c[1], c[2], c[3]);
                 part = dp4a_ss(w[p], 0x01010101u, part);
@@ -243,7 +243,7 @@ __device__ float quantise_row(const XT* __restrict__ row, int K, int Kp, int8_t*
 #pragma unroll
             for (int b = 0; b < 4; ++b) {
                 const int k = k4 + b;
-                c[b] = (k < K) ? __float2int_rn(__fmul_rn(xn(to_f(row[k]), k), s)) : 0;
+                c[b] = (k < K) ? (int)rint_low_byte(__fmul_rn(xn(to_f(row[k]), k), s)) : 0;
             }
             const uint32_t word = pack4(c[0], c[1], c[2], c[3]);
             *reinterpret_cast<uint32_t*>(q + k4) = word;

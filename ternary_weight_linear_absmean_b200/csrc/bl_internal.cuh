@@ -23,6 +23,16 @@ __host__ __device__ inline int64_t chunks_per_row(int64_t K) { return padded_k(K
 // bytes of one 8-row tile
 __host__ __device__ inline int64_t tile_bytes(int64_t K) { return chunks_per_row(K) * 8 * 16; }
 
+// ---- activation code rounding --------------------------------------------
+// rint(v), ties to even, for |v| <= 127.5, delivered in the low byte of a
+// float's bit pattern: adding 1.5 * 2^23 puts the sum in [2^23, 2^24), where
+// the fp32 spacing is 1, so the IEEE round-to-nearest-even addition rounds
+// v to an integer r (the constant is even, so ties go the way rint's do)
+// and the sum's bits are 0x4B400000 + r, whose low byte is r as an int8.
+// One addition on the FMA pipe in place of a float-to-int conversion, which
+// issues at a fraction of that rate; the caller packs the low bytes.
+__device__ __forceinline__ uint32_t rint_low_byte(float v) { return __float_as_uint(__fadd_rn(v, 12582912.0f)); }
+
 // ---- device status word bits --------------------------------------------
 constexpr unsigned kStatusNonfiniteW = 1u;
 constexpr unsigned kStatusNonfiniteX = 2u;
@@ -46,6 +56,25 @@ cudaError_t launch_quant(const void* x, bl_dtype xt, int64_t M, int64_t K, int8_
 // SubLN (RMS normalisation with gain [K], epsilon eps) then the quantiser.
 cudaError_t launch_rmsnorm_quant(const void* x, bl_dtype xt, const float* gain, double eps, int64_t M, int64_t K,
                                  int8_t* q, float* s, unsigned* status, cudaStream_t st);
+// The quantiser over the rows of several problems in one launch (one block
+// per row): problem i has rows [row_begin, row_begin + M) of the grid.
+struct QuantProblem {
+    const void* x;          // activations [M][K]
+    const float* gain;      // SubLN gain [K], or NULL
+    int8_t* q;              // [M][Kp]
+    float* s;               // [M]
+    int64_t K;
+    int row_begin;
+};
+constexpr int kMaxQuantGroup = 16;
+struct QuantBatch {
+    int row_begin[kMaxQuantGroup];   // copy of p[i].row_begin for the block -> problem search
+    QuantProblem p[kMaxQuantGroup];
+    int count;
+    int rows;               // total rows (the grid)
+    double eps;             // SubLN epsilon
+};
+cudaError_t launch_quant_grouped(const QuantBatch& b, bl_dtype xt, unsigned* status, cudaStream_t st);
 
 // One problem of the decode kernel (packed ternary x int8 -> y).
 struct GemvProblem {

@@ -10,13 +10,15 @@
 //   amax_m = max(max_k |x_mk|, 1e-5);  s_m = 127 / amax_m  (IEEE fp32 divide)
 //   q_mk   = clamp(rint(x_mk * s_m), -127, 127)          (fp32 multiply)
 //
-// One block per token row.  The row is read from memory once with 16-byte
+// One block per token row, over the rows of up to 16 problems (x, K, gain,
+// q, s each) in one launch.  The row is read from memory once with 16-byte
 // loads and kept in registers (up to 4 vectors per thread; longer rows are
 // re-read from L2).  Two exact shortcuts: max |x| is an unsigned max over
 // the bit patterns with the sign cleared (integer order is numeric order for
 // non-negative IEEE values, and NaN/Inf sort above every finite value, so
 // the same max flags non-finite input), and rint + clamp + convert is one
-// round-to-nearest-even conversion, since |x * s| < 127.5 for finite x.
+// round-to-nearest-even addition (rint_low_byte, bl_internal.cuh), since
+// |x * s| < 127.5 for finite x.
 // q rows have stride Kp = ceil(K/64)*64, zero-filled beyond K.  Built without
 // FMA contraction (-fmad=false) so every product rounds exactly once.
 #include "bl_internal.cuh"
@@ -83,18 +85,34 @@ __device__ __forceinline__ uint32_t block_reduce_max(uint32_t v, uint32_t* red)
     return t;
 }
 
+// A memory-bound kernel wants many warps per SM: bf16 rows without
+// normalisation fit 8 blocks (64 warps, 32 registers per thread); the other
+// forms need more registers and take 6 or 5 blocks without spilling.
 template <typename XT, bool NORM>
-__global__ void __launch_bounds__(kThreads)
-quant_kernel(const XT* __restrict__ x, int64_t K, int64_t Kp, const float* __restrict__ gain, double eps,
-             int8_t* __restrict__ q, float* __restrict__ s_out, unsigned* status)
+__global__ void __launch_bounds__(kThreads, NORM ? 5 : sizeof(XT) == 2 ? 8 : 6)
+quant_kernel(const __grid_constant__ QuantBatch b, unsigned* status)
 {
     __shared__ double redd[kWarps];
     __shared__ uint32_t redu[kWarps];
     using V = Vec<XT>;
     constexpr int E = V::E;
-    const int64_t m = blockIdx.x;
-    const XT* row = x + m * K;
-    int8_t* qrow = q + m * Kp;
+    int pi = 0;
+#pragma unroll 1
+    for (int i = 1; i < b.count; ++i)
+        if ((int)blockIdx.x >= b.row_begin[i]) pi = i;
+    const QuantProblem& P = b.p[pi];
+    const int64_t K = P.K, Kp = padded_k(P.K);
+    const float* __restrict__ gain = P.gain;
+    const double eps = b.eps;
+    const int64_t m = (int64_t)blockIdx.x - P.row_begin;
+    float* __restrict__ s_out = P.s;
+    // Programmatic dependent launch: a kernel launched after this one may
+    // start its own set-up now (it reads what this one writes only after
+    // its griddepcontrol.wait); this one reads nothing before its own wait.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    const XT* row = static_cast<const XT*>(P.x) + m * K;
+    int8_t* qrow = P.q + m * Kp;
     const int t = threadIdx.x;
     const bool vec = (K % E) == 0;
     const int64_t nv = K / E;
@@ -174,7 +192,7 @@ quant_kernel(const XT* __restrict__ x, int64_t K, int64_t Kp, const float* __res
                     int c[4];
 #pragma unroll
                     for (int b = 0; b < 4; ++b)
-                        c[b] = __float2int_rn(__fmul_rn(xn(V::get(u, 4 * p + b), v * E + 4 * p + b), s));
+                        c[b] = (int)rint_low_byte(__fmul_rn(xn(V::get(u, 4 * p + b), v * E + 4 * p + b), s));
                     w[p] = pack4(c[0], c[1], c[2], c[3]);
                 }
                 if constexpr (E == 8)
@@ -189,24 +207,53 @@ quant_kernel(const XT* __restrict__ x, int64_t K, int64_t Kp, const float* __res
 #pragma unroll
             for (int b = 0; b < 4; ++b) {
                 const int64_t k = k4 + b;
-                c[b] = (k < K) ? __float2int_rn(__fmul_rn(xn(load_x(row, k), k), s)) : 0;
+                c[b] = (k < K) ? (int)rint_low_byte(__fmul_rn(xn(load_x(row, k), k), s)) : 0;
             }
             *reinterpret_cast<uint32_t*>(qrow + k4) = pack4(c[0], c[1], c[2], c[3]);
         }
     }
 }
 
-template <typename XT>
-cudaError_t launch_typed(const void* x, int64_t M, int64_t K, const float* gain, double eps, int8_t* q, float* s,
-                         unsigned* status, cudaStream_t st)
+template <typename XT, bool NORM>
+cudaError_t launch_k(const QuantBatch& b, unsigned* status, cudaStream_t st)
 {
-    const int64_t Kp = padded_k(K);
-    const XT* xp = static_cast<const XT*>(x);
-    if (gain)
-        quant_kernel<XT, true><<<(unsigned)M, kThreads, 0, st>>>(xp, K, Kp, gain, eps, q, s, status);
-    else
-        quant_kernel<XT, false><<<(unsigned)M, kThreads, 0, st>>>(xp, K, Kp, nullptr, 0.0, q, s, status);
-    return cudaGetLastError();
+    // launched with programmatic stream serialisation: the kernel waits
+    // (griddepcontrol.wait) before it reads or writes anything
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)b.rows);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, quant_kernel<XT, NORM>, b, status);
+    return e != cudaSuccess ? e : cudaGetLastError();
+}
+
+template <typename XT>
+cudaError_t launch_typed(const QuantBatch& b, unsigned* status, cudaStream_t st)
+{
+    if (b.p[0].gain) return launch_k<XT, true>(b, status, st);
+    return launch_k<XT, false>(b, status, st);
+}
+
+QuantBatch single(const void* x, const float* gain, double eps, int64_t M, int64_t K, int8_t* q, float* s)
+{
+    QuantBatch b = {};
+    b.count = 1;
+    b.rows = (int)M;
+    b.eps = eps;
+    b.p[0].x = x;
+    b.p[0].gain = gain;
+    b.p[0].q = q;
+    b.p[0].s = s;
+    b.p[0].K = K;
+    b.p[0].row_begin = 0;
+    b.row_begin[0] = 0;
+    return b;
 }
 
 }  // namespace
@@ -214,15 +261,21 @@ cudaError_t launch_typed(const void* x, int64_t M, int64_t K, const float* gain,
 cudaError_t launch_quant(const void* x, bl_dtype xt, int64_t M, int64_t K, int8_t* q, float* s,
                          unsigned* status, cudaStream_t st)
 {
-    if (xt == BL_F32) return launch_typed<float>(x, M, K, nullptr, 0.0, q, s, status, st);
-    return launch_typed<__nv_bfloat16>(x, M, K, nullptr, 0.0, q, s, status, st);
+    return launch_quant_grouped(single(x, nullptr, 0.0, M, K, q, s), xt, status, st);
 }
 
 cudaError_t launch_rmsnorm_quant(const void* x, bl_dtype xt, const float* gain, double eps, int64_t M, int64_t K,
                                  int8_t* q, float* s, unsigned* status, cudaStream_t st)
 {
-    if (xt == BL_F32) return launch_typed<float>(x, M, K, gain, eps, q, s, status, st);
-    return launch_typed<__nv_bfloat16>(x, M, K, gain, eps, q, s, status, st);
+    return launch_quant_grouped(single(x, gain, eps, M, K, q, s), xt, status, st);
+}
+
+// Every problem of a batch either has a gain (SubLN) or none.
+cudaError_t launch_quant_grouped(const QuantBatch& b, bl_dtype xt, unsigned* status, cudaStream_t st)
+{
+    if (b.rows <= 0) return cudaSuccess;
+    if (xt == BL_F32) return launch_typed<float>(b, status, st);
+    return launch_typed<__nv_bfloat16>(b, status, st);
 }
 
 }  // namespace bl

@@ -172,15 +172,18 @@ __device__ __forceinline__ void quantise_rows(const XT* __restrict__ x, int M, i
         if (lane == 0 && m < M) atomicMax(&sh.amax[m], v);
     }
     sync();
+    // lane m of every warp divides for row m; the others take it by shuffle
+    // (one IEEE divide per thread rather than one per row)
     float s[MT];
+    {
+        const uint32_t bits = (lane < M) ? sh.amax[lane & 15] : 0u;
+        if (bits >= 0x7F800000u && tid < M) atomicOr(status, kStatusNonfiniteX);
+        const float mine = 127.0f / fmaxf(__uint_as_float(bits), 1e-5f);
 #pragma unroll
-    for (int m = 0; m < MT; ++m) {
-        const uint32_t bits = m < M ? sh.amax[m] : 0u;
-        if (bits >= 0x7F800000u && tid == 0) atomicOr(status, kStatusNonfiniteX);
-        s[m] = 127.0f / fmaxf(__uint_as_float(bits), 1e-5f);
+        for (int m = 0; m < MT; ++m) s[m] = __shfl_sync(0xffffffffu, mine, m);
     }
 
-    // ---- codes (one round-to-nearest-even conversion: |x * s| < 127.5)
+    // ---- codes (rint_low_byte: |x * s| < 127.5)
     //      and sum q per row
     int part[MT];
 #pragma unroll
@@ -201,7 +204,7 @@ __device__ __forceinline__ void quantise_rows(const XT* __restrict__ x, int M, i
                         for (int b = 0; b < 4; ++b) {
                             float e = elem(u[m], 4 * p + b);
                             if constexpr (NORM) e = __fmul_rn(__fmul_rn(e, r[m]), g[4 * p + b]);
-                            c[b] = __float2int_rn(__fmul_rn(e, s[m]));
+                            c[b] = (int)rint_low_byte(__fmul_rn(e, s[m]));
                         }
                         const uint32_t word = __byte_perm(__byte_perm(c[0], c[1], 0x0040),
                                                           __byte_perm(c[2], c[3], 0x0040), 0x5410);
@@ -219,7 +222,7 @@ __device__ __forceinline__ void quantise_rows(const XT* __restrict__ x, int M, i
 #pragma unroll
                     for (int b = 0; b < 4; ++b) {
                         const int k = 4 * kw + b;
-                        c[b] = (k < K) ? __float2int_rn(__fmul_rn(xn(xval(m, k), m, k), s[m])) : 0;
+                        c[b] = (k < K) ? (int)rint_low_byte(__fmul_rn(xn(xval(m, k), m, k), s[m])) : 0;
                     }
                     const uint32_t word = __byte_perm(__byte_perm(c[0], c[1], 0x0040),
                                                       __byte_perm(c[2], c[3], 0x0040), 0x5410);
@@ -236,7 +239,11 @@ __device__ __forceinline__ void quantise_rows(const XT* __restrict__ x, int M, i
     }
     sync();
     if (tid < M) {
-        s_out[tid] = 127.0f / fmaxf(__uint_as_float(sh.amax[tid]), 1e-5f);
+        float mine = s[0];
+#pragma unroll
+        for (int m = 1; m < MT; ++m)
+            if (tid == m) mine = s[m];
+        s_out[tid] = mine;
         sumq_out[tid] = sh.sumq[tid];
     }
 }

@@ -147,3 +147,35 @@ def test_rmsnorm_entries_reject_bad_arguments(L):
     assert g(2, arr, bl.BL_BF16, arr, 1e-6, arr, arr, 17, i64, i64, arr, bl.BL_F32, None) == bl.BL_ERR_SHAPE
     bad = (C.c_void_p * 2)(A, MIS)
     assert g(2, arr, bl.BL_BF16, bad, 1e-6, arr, arr, 1, i64, i64, arr, bl.BL_F32, None) == bl.BL_ERR_ALIGN
+
+
+def test_decode_workspace_bytes(L):
+    # per problem M * Kp bytes of codes and M fp32 scales, each rounded up
+    # to 256 bytes
+    f = L.bitlinear_decode_workspace_bytes
+    K2 = (C.c_int64 * 2)(64, 100)
+    assert f(2, 3, K2) == (256 + 256) + (512 + 256)
+    K1 = (C.c_int64 * 1)(11008)
+    assert f(1, 16, K1) == 16 * 11008 + 256
+    assert f(0, 3, K2) == 0 and f(17, 3, K2) == 0 and f(2, 0, K2) == 0 and f(2, 17, K2) == 0
+    assert f(2, 3, None) == 0
+    assert f(1, 1, (C.c_int64 * 1)(0)) == 0
+    assert f(1, 1, (C.c_int64 * 1)(16_909_321)) == 0
+
+
+def test_workspace_forms_reject_bad_workspaces(L):
+    # checked before any device work
+    g = L.bitlinear_forward_x_grouped_ws
+    arr = (C.c_void_p * 2)(A, A)
+    i64 = (C.c_int64 * 2)(8, 64)
+    need = L.bitlinear_decode_workspace_bytes(2, 4, i64)
+    assert need > 0
+    assert g(2, arr, bl.BL_BF16, arr, arr, 4, i64, i64, arr, bl.BL_F32, None, need, None) == bl.BL_ERR_NULL
+    assert g(2, arr, bl.BL_BF16, arr, arr, 4, i64, i64, arr, bl.BL_F32, MIS, need, None) == bl.BL_ERR_ALIGN
+    assert g(2, arr, bl.BL_BF16, arr, arr, 4, i64, i64, arr, bl.BL_F32, A, need - 1, None) == bl.BL_ERR_WORKSPACE
+    assert g(2, arr, bl.BL_BF16, arr, arr, 17, i64, i64, arr, bl.BL_F32, A, need, None) == bl.BL_ERR_SHAPE
+    h = L.bitlinear_forward_x_rmsnorm_grouped_ws
+    assert h(2, arr, bl.BL_BF16, None, 1e-6, arr, arr, 4, i64, i64, arr, bl.BL_F32, A, need, None) == bl.BL_ERR_NULL
+    assert h(2, arr, bl.BL_BF16, arr, -1.0, arr, arr, 4, i64, i64, arr, bl.BL_F32, A, need, None) == bl.BL_ERR_ARG
+    assert h(2, arr, bl.BL_BF16, arr, 1e-6, arr, arr, 4, i64, i64, arr, bl.BL_F32, A, need - 1,
+             None) == bl.BL_ERR_WORKSPACE

@@ -253,3 +253,79 @@ def test_grouped_mixed_ring_depths(bl, M):
     for y, ref in zip(ys, refs):
         P.check_y_f32(y.cpu().numpy(), ref["y"], exact=True)
 
+
+
+@pytest.mark.parametrize("M", [1, 2, 3, 8, 16])
+def test_workspace_form(bl, kind, M):
+    # quantise-once launch + product on the codes (M >= 2): the same y, bit
+    # for bit, as the single-launch form and the oracle; the workspace is
+    # reused by a second call
+    import torch
+    shapes = [(640, 2560), (96, 4097), (300, 1000), (8, 64)]
+    xs, ps, gs, y1, y2, refs = [], [], [], [], [], []
+    for i, (N, K) in enumerate(shapes):
+        W = synth.weights(N, K, seed=1100 + i)
+        x = synth.activations(M, K, seed=1200 + i + M, dtype="bf16", outlier_frac=0.01)
+        refs.append(oracle.bitlinear(W, x, "bf16"))
+        p, _, g = _packed(bl, W)
+        xs.append(P.to_dev_bf16(x))
+        ps.append(p)
+        gs.append(g)
+        y1.append(torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda"))
+        y2.append(torch.empty((M, N), dtype=torch.float32, device="cuda"))
+    Ns, Ks = [s[0] for s in shapes], [s[1] for s in shapes]
+    ws = bl.decode_workspace(M, Ks, "cuda")
+    bl.bitlinear_forward_x_grouped(xs, ps, gs, Ns, Ks, y1, workspace=ws)
+    bl.bitlinear_forward_x_grouped(xs, ps, gs, Ns, Ks, y1, workspace=ws)
+    bl.bitlinear_forward_x_grouped(xs, ps, gs, Ns, Ks, y2)
+    torch.cuda.synchronize()
+    assert bl.bitlinear_get_status() == bl.BL_OK
+    for a, b, ref in zip(y1, y2, refs):
+        assert np.array_equal(a.cpu().numpy(), b.cpu().numpy())
+        P.check_y_f32(a.cpu().numpy(), ref["y"], exact=True)
+
+
+@pytest.mark.parametrize("M", [4, 16])
+def test_workspace_form_beyond_the_streaming_limit(bl, M):
+    import torch
+    shapes = [(200, 11008), (128, 4096)]
+    xs, ps, gs, ys, refs = [], [], [], [], []
+    for i, (N, K) in enumerate(shapes):
+        W = synth.weights(N, K, seed=1300 + i)
+        x = synth.activations(M, K, seed=1400 + i, dtype="f32", outlier_frac=0.01)
+        refs.append(oracle.bitlinear(W, x, "f32"))
+        p, _, g = _packed(bl, W)
+        xs.append(P.to_dev_f32(x))
+        ps.append(p)
+        gs.append(g)
+        ys.append(torch.empty((M, N), dtype=torch.bfloat16, device="cuda"))
+    Ns, Ks = [s[0] for s in shapes], [s[1] for s in shapes]
+    bl.bitlinear_forward_x_grouped(xs, ps, gs, Ns, Ks, ys, workspace=bl.decode_workspace(M, Ks, "cuda"))
+    torch.cuda.synchronize()
+    assert bl.bitlinear_get_status() == bl.BL_OK
+    for y, ref in zip(ys, refs):
+        assert np.array_equal(P.bf16_dev_to_bits(y), oracle.to_bf16(ref["y"]))
+
+
+def test_prepared_grouped_call_with_gains(bl):
+    # GroupedDecode with gains: the SubLN workspace form, equal to the plain
+    # SubLN grouped call
+    import torch
+    M, eps, shapes = 5, 1e-6, [(640, 2560), (96, 4097)]
+    xs, gains, ps, gs, y1, y2 = [], [], [], [], [], []
+    for i, (N, K) in enumerate(shapes):
+        W = synth.weights(N, K, seed=1500 + i)
+        xs.append(P.to_dev_bf16(synth.activations(M, K, seed=1600 + i, dtype="bf16")))
+        gains.append(P.to_dev_f32((1.0 + 0.25 * np.random.default_rng(K).standard_normal(K)).astype(np.float32)))
+        p, _, g = _packed(bl, W)
+        ps.append(p)
+        gs.append(g)
+        y1.append(torch.empty((M, N), dtype=torch.float32, device="cuda"))
+        y2.append(torch.empty((M, N), dtype=torch.float32, device="cuda"))
+    Ns, Ks = [s[0] for s in shapes], [s[1] for s in shapes]
+    bl.GroupedDecode(xs, ps, gs, Ns, Ks, y1, gains=gains, eps=eps)()
+    bl.bitlinear_forward_x_rmsnorm_grouped(xs, gains, eps, ps, gs, Ns, Ks, y2)
+    torch.cuda.synchronize()
+    assert bl.bitlinear_get_status() == bl.BL_OK
+    for a, b in zip(y1, y2):
+        assert np.array_equal(a.cpu().numpy(), b.cpu().numpy())

@@ -162,3 +162,38 @@ def test_rmsnorm_grouped_beyond_the_streaming_limit(bl):
     assert all(straddle_rows(x, "bf16", eps).sum() == 0 for x in xs_host)
     for y, ref in zip(ys, refs):
         P.check_y_f32(y.cpu().numpy(), ref["y"], exact=True)
+
+
+@pytest.mark.parametrize("kind", ["auto", "tensor", "dp4a", "tile"])
+@pytest.mark.parametrize("M", [2, 16])
+def test_rmsnorm_workspace_form(bl, kind, M):
+    # SubLN quantised once per row (grouped quantiser launch), then the
+    # product on the codes: against the oracle, every decode kernel
+    import torch
+    eps = 1e-6
+    shapes = [(640, 2560), (96, 4097), (8, 64)]
+    xs, gains, ps, gs, ys, refs, xs_host = [], [], [], [], [], [], []
+    for i, (N, K) in enumerate(shapes):
+        W = synth.weights(N, K, seed=1700 + i)
+        x = synth.activations(M, K, seed=1800 + i, dtype="bf16", outlier_frac=0.01)
+        g = _gain(K, 1900 + i)
+        refs.append(oracle.bitlinear_rmsnorm(W, x, "bf16", g, eps))
+        p, _, g32 = bl.pack(P.to_dev_f32(W))
+        xs.append(P.to_dev_bf16(x))
+        xs_host.append(x)
+        gains.append(P.to_dev_f32(g))
+        ps.append(p)
+        gs.append(g32)
+        ys.append(torch.empty((M, N), dtype=torch.float32, device="cuda"))
+    Ns, Ks = [s[0] for s in shapes], [s[1] for s in shapes]
+    bl.bitlinear_set_decode_kernel({"tile": bl.BL_DECODE_TILE}.get(kind, KINDS.get(kind)))
+    try:
+        bl.bitlinear_forward_x_rmsnorm_grouped(xs, gains, eps, ps, gs, Ns, Ks, ys,
+                                               workspace=bl.decode_workspace(M, Ks, "cuda"))
+        torch.cuda.synchronize()
+    finally:
+        bl.bitlinear_set_decode_kernel(bl.BL_DECODE_AUTO)
+    assert bl.bitlinear_get_status() == bl.BL_OK
+    assert all(straddle_rows(x, "bf16", eps).sum() == 0 for x in xs_host)
+    for y, ref in zip(ys, refs):
+        P.check_y_f32(y.cpu().numpy(), ref["y"], exact=True)
