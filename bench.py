@@ -145,7 +145,7 @@ def decode_bytes(lin, M):
 # entry to None when that kernel changes.
 MEASURED_TRAFFIC = {
     # stream_kernel<1, fused, bf16, fp32, 4>, 2B block, M = 1, grouped launch
-    ("block2b", "stream_kernel", 1): 17_471_744,
+    ("block2b", "stream_kernel", 1): 17_469_184,
     # gemm_tc_kernel<bf16>, M = 2048: mean of the step's two launches
     # (2560->6912: 9,722,368 B; 6912->2560: 18,645,504 B)
     ("prefill", "gemm_tc_kernel", 2048): 14_183_936,
@@ -718,7 +718,7 @@ def main():
             ems, n, hb, db = run_e2e(torch, bl, lin, M, dev, stream, R["S"], args.steps, dist)
             out["e2e"] = {"value": nbytes * n * world / (ems / 1e3) / 1e9, "unit": "GB/s",
                           "h2d_bytes_per_step": hb, "d2h_bytes_per_step": db, "ms_per_step": ems / n,
-                          "path": "pinned host x -> H2D -> bitlinear_forward_x_grouped (C ABI, prepared "
+                          "path": "pinned host x -> H2D -> bitlinear_forward_x_grouped_ws (C ABI, prepared "
                                   "GroupedDecode call) -> D2H y"}
         if args.workload == "block2b" and not args.no_prefill:
             out["prefill"] = run_prefill(torch, bl, args, dev, stream, dist, l2, 20)
