@@ -264,9 +264,12 @@ bl_status bitlinear_forward_x_grouped(int count, const void* const* x, bl_dtype 
                                       void* const* y, bl_dtype yt, void* stream);
 
 /* ------------------------------------------------------------------------
- * Workspace forms of the grouped fused decode calls.  Same arguments,
- * results (bit for bit) and errors as bitlinear_forward_x_grouped and
- * bitlinear_forward_x_rmsnorm_grouped, plus a device workspace (16-byte
+ * Workspace forms of the grouped fused decode calls: the same layer
+ * (aratech.ae, "BitLinear: the building block": per-token absmax int8
+ * activations, ternary weights, rescale), the same arguments, results (bit
+ * for bit) and errors as bitlinear_forward_x_grouped and
+ * bitlinear_forward_x_rmsnorm_grouped -- except that under BL_DECODE_TILE
+ * the SubLN form runs for M >= 2 (on the codes) -- plus a device workspace (16-byte
  * aligned, caller-owned, at least bitlinear_decode_workspace_bytes(count,
  * M, K) bytes, else BL_ERR_WORKSPACE; NULL: BL_ERR_NULL) that the call may
  * overwrite, in stream order.  For M >= 2 the call quantises every token
