@@ -157,6 +157,34 @@ def test_block2b_grouped_single_launch(bl):
         P.check_y_f32(y.cpu().numpy(), ref["y"], exact=True)
 
 
+@pytest.mark.parametrize("M", synth.M_7B)
+def test_7b_group_as_benched(bl, M):
+    # the 7B-class decode step exactly as bench.py times it: the three
+    # linears' inputs from the same seeds, one prepared grouped call
+    # (workspace form: for M >= 2 a quantiser launch, then the product on the
+    # codes), every output element against the oracle
+    import torch
+    xs, ps, gs, ys, refs, Ns, Ks = [], [], [], [], [], [], []
+    for i, (K, N, _) in enumerate(synth.SHAPES_7B):
+        W = synth.weights(N, K, 10 + i)
+        x = synth.activations(M, K, 2000 + i, "bf16")
+        refs.append(oracle.bitlinear(W, x, "bf16"))
+        packed, _, g32 = bl.pack(P.to_dev_f32(W))
+        xs.append(P.to_dev_bf16(x))
+        ps.append(packed)
+        gs.append(g32)
+        ys.append(torch.empty((M, N), dtype=torch.float32, device="cuda"))
+        Ns.append(N)
+        Ks.append(K)
+    step = bl.GroupedDecode(xs, ps, gs, Ns, Ks, ys)
+    step()
+    step()
+    torch.cuda.synchronize()
+    assert bl.bitlinear_get_status() == bl.BL_OK
+    for y, ref in zip(ys, refs):
+        P.check_y_f32(y.cpu().numpy(), ref["y"], exact=True)
+
+
 @pytest.mark.parametrize("K,N", [(K, N) for K, N, _ in synth.SHAPES_7B])
 @pytest.mark.parametrize("M", synth.M_7B)
 def test_7b_shapes_full(bl, M, K, N):
