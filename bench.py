@@ -16,7 +16,9 @@ HBM.  Steps are replayed from CUDA graphs and timed with CUDA events on the
 launching stream; multi-GPU runs are independent replicas (no collective on
 the data path), timed as the max over ranks.
 
-Other workloads (--workload): 7b (decode at 7B-class shapes, --m 1/4/16),
+Other workloads (--workload): 7b (decode at 7B-class shapes, --m 1/4/16; from
+two tokens up a step is the grouped call's workspace form: one quantiser
+launch over the three linears, then one product launch on the codes),
 prefill (M = 2048 tokens on the tensor cores; metric int8 TOPS), pack
 (absmean quantise + 2-bit pack of the block's weights), sweep100b (one token
 through 80 layers x 7 linears of a 100B-class model, 17.1 GB of packed
